@@ -1,0 +1,280 @@
+"""Pins for the oracle: each check is fixed by the GPTQ pages or by mathematics, not by the oracle.
+
+A plausible mistake anywhere in the oracle (a dropped term, a wrong sign or index, a transposed
+operand, quantizing the original instead of the compensated value) fails at least one of these;
+``test_planted_mistakes_are_caught`` plants such mistakes on the CPU and checks that.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+from conftest import read_golden
+
+
+def _spd(d, rng, cond=50.0):
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    ev = np.geomspace(1.0, cond, d)
+    return (Q * ev) @ Q.T
+
+
+def _correlated_x(n, d, rng):
+    return rng.standard_normal((n, d)) @ (rng.standard_normal((d, d)) / np.sqrt(d))
+
+
+# ------------------------------------------------------------------------------------ A1 / A2
+def test_hessian_worked_example(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "hessian_example.txt"))
+    X = np.array(g["x"], dtype=float).reshape(3, 2)
+    np.testing.assert_array_equal(O.hessian(X), np.array(g["h"], dtype=float).reshape(2, 2))
+    np.testing.assert_allclose(O.dampen(O.hessian(X), 0.01),
+                               np.array(g["hd"], dtype=float).reshape(2, 2), rtol=0, atol=1e-12)
+
+
+def test_hessian_is_sum_of_token_outer_products():
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((37, 9))
+    H = np.zeros((9, 9))
+    for t in range(37):  # brute force, one token at a time
+        for i in range(9):
+            for j in range(9):
+                H[i, j] += 2.0 * X[t, i] * X[t, j]
+    np.testing.assert_allclose(O.hessian(X), H, rtol=1e-13, atol=1e-12)
+    Hc = np.zeros((9, 9))
+    for c0 in range(0, 37, 8):  # accumulation over token chunks is additive
+        O.hessian_accumulate(Hc, X[c0:c0 + 8])
+    np.testing.assert_allclose(Hc, H, rtol=1e-13, atol=1e-12)
+
+
+def test_dampen_adds_fraction_of_mean_diagonal():
+    H = np.diag([1.0, 2.0, 3.0, 6.0]) + 0.5
+    Hd = O.dampen(H, 0.01)
+    lam = 0.01 * np.mean([1.5, 2.5, 3.5, 6.5])
+    np.testing.assert_allclose(np.diag(Hd) - np.diag(H), lam)
+    off = ~np.eye(4, dtype=bool)
+    np.testing.assert_array_equal(Hd[off], H[off])
+
+
+# ------------------------------------------------------------------------------------ A3
+@pytest.mark.parametrize("d", [1, 2, 7, 40, 130])
+def test_upper_factor_of_inverse(d):
+    rng = np.random.default_rng(d)
+    Hd = _spd(d, rng, cond=1e3)
+    U = O.inverse_upper_cholesky(Hd)
+    assert np.allclose(np.tril(U, -1), 0.0)
+    assert np.all(np.diag(U) > 0)
+    # U^T U = Hd^-1  <=>  U Hd U^T = I (U invertible); no inverse needed on this side
+    res = np.linalg.norm(U @ Hd @ U.T - np.eye(d)) / np.sqrt(d)
+    assert res < 1e-10
+    np.testing.assert_allclose(O.inverse_upper_cholesky_reversed(Hd), U, rtol=1e-8, atol=1e-10)
+
+
+def test_upper_factor_worked_example(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "worked_example_d3.txt"))
+    Hd = np.array(g["hd"], dtype=float).reshape(3, 3)
+    U = O.inverse_upper_cholesky(Hd)
+    np.testing.assert_allclose(np.diag(U), np.array(g["u_diag"], dtype=float), rtol=1e-14)
+    np.testing.assert_allclose(U[0, 1] / U[0, 0], -2.0 / 3.0, rtol=1e-14)
+    np.testing.assert_allclose(U[0, 2] / U[0, 0], 1.0 / 3.0, rtol=1e-14)
+    np.testing.assert_allclose(U[1, 2] / U[1, 1], -0.5, rtol=1e-14)
+
+
+# ------------------------------------------------------------------------------------ A4 grid
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_grid_is_a_uniform_asymmetric_quantizer(bits):
+    rng = np.random.default_rng(bits)
+    maxq = 2 ** bits - 1
+    for _ in range(200):
+        x = rng.standard_normal(64) * rng.uniform(0.01, 3.0) + rng.uniform(-1, 1)
+        s, z = O.grid_params(x.min(), x.max(), bits)
+        lo, hi = min(0.0, x.min()), max(0.0, x.max())
+        assert 0 <= z <= maxq
+        q = O.quantize_codes(x, s, z, bits)
+        assert q.min() >= 0 and q.max() <= maxq
+        assert O.dequantize(z, s, z) == 0.0          # zero is exactly representable
+        np.testing.assert_allclose(s, (hi - lo) / maxq, rtol=1e-6)
+        # every value of the range lies within half a step (plus the zero-point shift) of its level
+        err = np.abs(O.dequantize(q, s, z) - x)
+        assert err.max() <= s * 1.0 + 1e-6
+        # an all-zero range falls back to [-1, 1]
+    s, z = O.grid_params(0.0, 0.0, bits)
+    np.testing.assert_allclose(s, 2.0 / maxq, rtol=1e-7)
+
+
+def test_grid_in_range_error_is_half_step_for_symmetric_endpoints():
+    # when -xmin/scale is an integer the grid contains both endpoints and rounding error <= scale/2
+    s, z = O.grid_params(-0.3, 0.6, 2)  # scale 0.3, zero 1 -> levels -0.3, 0, 0.3, 0.6
+    assert z == 1
+    x = np.linspace(-0.3, 0.6, 1001)
+    err = np.abs(O.dequantize(O.quantize_codes(x, s, z, 2), s, z) - x)
+    assert err.max() <= 0.15 + 1e-6
+
+
+# ------------------------------------------------------------------------------------ A5 / A6
+def test_worked_example_d3(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "worked_example_d3.txt"))
+    Hd = np.array(g["hd"], dtype=float).reshape(3, 3)
+    w = np.array(g["w"], dtype=float)[None, :]
+    bits = int(g["bits"][0])
+    U = O.inverse_upper_cholesky(Hd)
+    r = O.gptq_quantize(w, U, bits)
+    np.testing.assert_array_equal(r["codes"][0], np.array(g["codes"], dtype=int))
+    np.testing.assert_allclose(r["Err"][0], np.array(g["err"], dtype=float), rtol=1e-6)
+    comp = r["Wq"][0] + r["Err"][0] * np.diag(U)  # compensated value = deq + delta
+    np.testing.assert_allclose(comp, np.array(g["compensated"], dtype=float), rtol=1e-6)
+    np.testing.assert_array_equal(O.rtn_quantize(w, bits)["codes"][0],
+                                  np.array(g["rtn_codes"], dtype=int))
+
+
+@pytest.mark.parametrize("group_size", [0, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_diagonal_hessian_reduces_to_rtn(bits, group_size):
+    """H proportional to I (or any diagonal H): U is diagonal, no error is propagated, and GPTQ's
+    codes are round-to-nearest's on the same grid."""
+    rng = np.random.default_rng(10 * bits + group_size)
+    W = rng.standard_normal((16, 32)) * 0.02
+    for Hd in (3.7 * np.eye(32), np.diag(rng.uniform(0.5, 5.0, 32))):
+        U = O.inverse_upper_cholesky(Hd)
+        assert np.allclose(U, np.diag(np.diag(U)))
+        g = O.gptq_quantize(W, U, bits, group_size, block_size=8)
+        r = O.rtn_quantize(W, bits, group_size)
+        np.testing.assert_array_equal(g["codes"], r["codes"])
+        np.testing.assert_array_equal(g["scales"], r["scales"])
+        np.testing.assert_array_equal(g["zeros"], r["zeros"])
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("group_size", [0, 4])
+def test_cholesky_form_equals_explicit_obs(seed, group_size):
+    rng = np.random.default_rng(seed)
+    d = 16
+    X = _correlated_x(64, d, rng)
+    Hd = O.dampen(O.hessian(X), 0.01)
+    W = rng.standard_normal((12, d)) * 0.02
+    g = O.gptq_quantize(W, O.inverse_upper_cholesky(Hd), 3, group_size)
+    o = O.obs_quantize(W, Hd, 3, group_size)
+    np.testing.assert_array_equal(g["codes"], o["codes"])
+    np.testing.assert_allclose(g["scales"], o["scales"], rtol=1e-6)
+    np.testing.assert_array_equal(g["zeros"], o["zeros"])
+
+
+@pytest.mark.parametrize("d,bits", [(3, 4), (4, 3), (5, 2), (6, 2), (6, 3)])
+def test_greedy_matches_conditional_least_squares_and_bruteforce(d, bits):
+    """(i) After any prefix of columns is fixed, the compensated remaining values are the
+    least-squares optimum of the layer objective given that prefix; (ii) the exhaustive optimum over
+    all code vectors is no worse than the greedy result or round-to-nearest."""
+    rng = np.random.default_rng(100 * d + bits)
+    for trial in range(4):
+        X = _correlated_x(32, d, rng)
+        Hd = O.dampen(O.hessian(X), 0.01)
+        U = O.inverse_upper_cholesky(Hd)
+        w = rng.standard_normal((1, d)) * 0.02
+        r = O.gptq_quantize(w, U, bits)
+        comp = r["Wq"][0] + r["Err"][0] * np.diag(U)
+        for k in range(1, d):
+            v = O.conditional_ls_values(w[0], Hd, r["Wq"][0, :k])
+            np.testing.assert_allclose(comp[k], v[0], rtol=1e-9, atol=1e-12)
+        s, z = r["scales"][0, 0], r["zeros"][0, 0]
+        qbest, obest = O.bruteforce_best_codes(w[0], Hd, bits, s, z)
+        dg = w[0] - r["Wq"][0]
+        ogreedy = dg @ Hd @ dg
+        dr = w[0] - O.rtn_quantize(w, bits)["Wq"][0]
+        assert obest <= ogreedy * (1 + 1e-12) + 1e-18
+        assert obest <= dr @ Hd @ dr * (1 + 1e-12) + 1e-18
+
+
+def test_gptq_beats_rtn_statistic():
+    """Expected statistic (the pages: GPTQ beats round-to-nearest at 3-4 bits because correlated
+    inputs let other weights absorb the error): on the tiny correlated layer shape, the layer
+    reconstruction error is at most RTN's in at least 95 of 100 seeded trials."""
+    wins = 0
+    for seed in range(100):
+        rng = np.random.default_rng(seed)
+        W = rng.standard_normal((64, 128)) * 0.02
+        Z = rng.standard_normal((256, 128))
+        A = rng.standard_normal((128, 128)) / np.sqrt(128)
+        X = Z @ A
+        res = O.gptq_layer(W, X, bits=4, group_size=0, block_size=32)
+        e_rtn = O.reconstruction_error(W, O.rtn_quantize(W, 4)["Wq"], res["H"])
+        wins += res["E"] <= e_rtn
+    assert wins >= 95
+
+
+@pytest.mark.parametrize("group_size", [0, 8, 32])
+def test_blocking_and_scaling_do_not_change_codes(group_size):
+    rng = np.random.default_rng(7 + group_size)
+    d = 64
+    X = _correlated_x(128, d, rng)
+    H = O.hessian(X)
+    W = rng.standard_normal((20, d)) * 0.02
+    U = O.inverse_upper_cholesky(O.dampen(H, 0.01))
+    ref = O.gptq_quantize(W, U, 3, group_size, block_size=0)
+    for B in (1, 4, 32):
+        if group_size and group_size % B and B % group_size:
+            continue
+        r = O.gptq_quantize(W, U, 3, group_size, block_size=B)
+        np.testing.assert_array_equal(r["codes"], ref["codes"])
+        np.testing.assert_allclose(r["Wq"], ref["Wq"], rtol=0, atol=1e-12)
+    # H -> c H (the pages' H = 2XX^T versus X^T X / N): damping scales along, codes are unchanged
+    Us = O.inverse_upper_cholesky(O.dampen(H * 1e-3 / len(X), 0.01))
+    r = O.gptq_quantize(W, Us, 3, group_size, block_size=16 if group_size != 8 else 8)
+    np.testing.assert_array_equal(r["codes"], ref["codes"])
+
+
+def test_reconstruction_error_two_forms():
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((50, 12))
+    W = rng.standard_normal((5, 12))
+    Wq = W + 0.01 * rng.standard_normal((5, 12))
+    direct = np.sum(((W - Wq) @ X.T) ** 2)
+    np.testing.assert_allclose(O.reconstruction_error(W, Wq, O.hessian(X)), direct, rtol=1e-12)
+
+
+# ------------------------------------------------------------------------------------ A7 pack
+def test_pack_hand_worked_examples(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "pack_examples.txt"))
+    for row in g["rows"]:
+        bits, n, period = int(row[0]), int(row[1]), int(row[2])
+        words = np.array([int(h, 16) for h in row[3:]], dtype=np.uint64).astype(np.uint32)
+        codes = (np.arange(n) % period)[None, :]
+        packed = O.pack_codes(codes, bits)
+        np.testing.assert_array_equal(packed.view(np.uint32)[0], words)
+        np.testing.assert_array_equal(O.unpack_codes(packed, bits, n), codes)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_roundtrip(bits):
+    rng = np.random.default_rng(bits)
+    codes = rng.integers(0, 2 ** bits, size=(7, 96))
+    p = O.pack_codes(codes, bits)
+    assert p.shape == (7, 96 * bits // 32) and p.dtype == np.int32
+    np.testing.assert_array_equal(O.unpack_codes(p, bits, 96), codes)
+
+
+# ------------------------------------------------------------------------------------ mutation check
+def test_planted_mistakes_are_caught():
+    """Plant plausible mistakes in what the column loop is given and check a pin fails for each."""
+    rng = np.random.default_rng(11)
+    d = 12
+    X = _correlated_x(48, d, rng)
+    Hd = O.dampen(O.hessian(X), 0.01)
+    W = rng.standard_normal((16, d)) * 0.05
+    U = O.inverse_upper_cholesky(Hd)
+    obs = O.obs_quantize(W, Hd, 3)["codes"]
+    assert np.array_equal(O.gptq_quantize(W, U, 3)["codes"], obs)
+    Uo = U - np.diag(np.diag(U))
+    mistakes = {
+        "transposed U": U.T,
+        "wrong sign of the update": np.diag(np.diag(U)) - Uo,
+        "dropped division by U_ii": Uo + np.eye(d),
+        "Cholesky of H instead of its inverse": np.linalg.cholesky(Hd).T,
+        "no compensation": np.diag(np.diag(U)),
+    }
+    for name, Ubad in mistakes.items():
+        caught = False
+        try:
+            caught = not np.array_equal(O.gptq_quantize(W, Ubad, 3)["codes"], obs)
+        except Exception:
+            caught = True
+        assert caught, name
