@@ -1,0 +1,167 @@
+/*
+ * gptq.h — C ABI of the GPTQ layer-wise quantization solver for NVIDIA B200 (sm_100a).
+ *
+ * GPTQ (Frantar, Ashkboos, Hoefler, Alistarh; ICLR 2023) quantizes one linear layer W[out, in] at a
+ * time so that the layer's output on calibration inputs X[tokens, in] changes as little as possible
+ * (FDE Interviews breakdown of GPTQ, section 01 "The paper in one minute"; zhiliyouxian blog
+ * "GPTQ：用于生成式预训练 Transformer 的准确训练后量化", section 数学基础 and the layer routine in
+ * 算法流程, whose arguments are W [out_features, in_features], X [batch, in_features], bits).
+ *
+ * The solver runs in four calls, in this order:
+ *   1. gptq_hessian_accumulate   H  = 2 X^T X                      (A1)
+ *   2. gptq_prepare_uinv         Hd = H + damp*mean(diag H)*I;  U = chol(Hd^-1), upper   (A2, A3)
+ *   3. gptq_quantize_layer       column loop + lazy block updates -> codes, scales, zeros (A4-A6)
+ *   4. gptq_pack                 b-bit codes -> int32 words                                (A7)
+ *
+ * Conventions shared by every entry point:
+ *  - Matrices are dense and row-major with no padding (leading dimension = number of columns).
+ *  - Every pointer argument except `cfg` and `detail` is DEVICE memory on the current CUDA device,
+ *    allocated and owned by the caller.  The library allocates no device or host memory and keeps no
+ *    state between calls (apart from a cached driver entry point).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues work on
+ *    that stream and returns; results are ready when the stream reaches that point.
+ *  - Arguments are validated on the host before anything is enqueued; a bad argument returns
+ *    GPTQ_ERR_ARG (or GPTQ_ERR_UNSUPPORTED / GPTQ_ERR_WORKSPACE) and enqueues nothing.
+ *  - Failures found on the device (a non-positive pivot, a bounded wait that gave up) are written
+ *    to the caller's device status word `dev_status` (int32[2]: code, detail), never trapped; read it
+ *    with gptq_read_status.  Kernels never spin without an iteration limit.
+ *  - A launch failure returns GPTQ_ERR_CUDA.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPTQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GPTQ_API __attribute__((visibility("default")))
+#else
+#define GPTQ_API
+#endif
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_ARG = 1,          /* null pointer, bad size, misaligned pointer, bad combination    */
+  GPTQ_ERR_UNSUPPORTED = 2,  /* a valid option this library does not implement (act-order)    */
+  GPTQ_ERR_NOT_PD = 3,       /* device: the dampened Hessian is not positive definite          */
+  GPTQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed                           */
+  GPTQ_ERR_TIMEOUT = 5,      /* device: a bounded wait inside a kernel gave up                 */
+  GPTQ_ERR_WORKSPACE = 6     /* workspace pointer null or smaller than the *_workspace_size    */
+} gptq_status;
+
+typedef enum { GPTQ_BF16 = 0, GPTQ_FP16 = 1, GPTQ_FP32 = 2 } gptq_dtype;
+
+/* Flags of gptq_quant_cfg.flags. */
+#define GPTQ_FLAG_ACT_ORDER 1u /* reorder columns by descending diag(H) ("desc_act"); unsupported */
+
+/* Quantization settings of one layer (zhiliyouxian blog, 实践指南: bits, group_size, desc_act;
+ * agent.csdn.net "GPTQ量化参数搜索工具", 关键参数说明 table: bits, group_size, zero point;
+ * FDE breakdown figure step 4: blocks of 128 columns). */
+typedef struct {
+  int32_t bits;        /* 2, 3 or 4: codes lie in [0, 2^bits - 1]                                 */
+  int32_t group_size;  /* 0: one grid per row; else a multiple of 32 that divides d, and either
+                          group_size divides block_size or block_size divides group_size         */
+  int32_t block_size;  /* columns per lazy-update block: 32, 64 or 128                            */
+  uint32_t flags;      /* GPTQ_FLAG_* ; 0 for the plain method                                    */
+} gptq_quant_cfg;
+
+/* ------------------------------------------------------------------------------------------
+ * A1  H = accumulate ? H + scale * X^T X : scale * X^T X
+ *
+ * The curvature of the layer-wise least-squares objective, H = 2 X X^T with X as [in, tokens]
+ * (FDE breakdown, section 01 and figure "THE IDEA, VISUALLY"); here X is [tokens, in] so H = 2 X^T X
+ * and `scale` = 2 reproduces the pages.  The sum over tokens is additive, so a caller may feed the
+ * calibration set in chunks with accumulate = 1.
+ *
+ *   X          [n_tokens, d] row-major, dtype x_dtype (BF16 / FP16 use the tensor cores with fp32
+ *              accumulation; FP32 uses fp32 FMA).  Must be 16-byte aligned.
+ *   H          [d, d] fp32 row-major.  On return the upper triangle (j >= i) holds the result; the
+ *              strict lower triangle is left unspecified.
+ *   workspace  >= gptq_hessian_workspace_size(n_tokens, d, x_dtype) bytes, 256-byte aligned.
+ *   dev_status int32[2] device status word (written only on a device-side failure).
+ *   Requires d % 8 == 0, n_tokens >= 0 (0 tokens gives H = 0 or leaves H unchanged).
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_hessian_accumulate(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d,
+                                    float* H, float scale, int32_t accumulate, int32_t* dev_status,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+GPTQ_API size_t gptq_hessian_workspace_size(int64_t n_tokens, int64_t d, int32_t x_dtype);
+
+/* ------------------------------------------------------------------------------------------
+ * A2 + A3  U = upper Cholesky factor of (H + damp * mean(diag H) * I)^-1
+ *
+ * Dampening: zhiliyouxian blog 算法流程 ("H = H + lambda * I") and 实践指南 (damp_percent = 0.01);
+ * nubint.ai review, "Proposed method" (Cholesky reformulation and dampening for stability).
+ * U: FDE breakdown figure step 2 ("U = chol(H^-1)") and section 01 (rows of the inverse Hessian
+ * from a Cholesky decomposition).  U^T U = Hd^-1, U upper with positive diagonal.
+ *
+ *   H          [d, d] fp32, upper triangle read (as written by gptq_hessian_accumulate); unchanged.
+ *   U          [d, d] fp32 output: upper triangle = the factor, strict lower triangle = 0.
+ *              Also used as scratch during the call; must not alias H.
+ *   dev_status int32[2]: cleared at the start of the call; {GPTQ_ERR_NOT_PD, pivot column} if the
+ *              dampened matrix is not positive definite (U is then unspecified).
+ *   workspace  >= gptq_prepare_workspace_size(d) bytes, 256-byte aligned.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_prepare_uinv(const float* H, int64_t d, float damp, float* U, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, void* stream);
+GPTQ_API size_t gptq_prepare_workspace_size(int64_t d);
+
+/* ------------------------------------------------------------------------------------------
+ * A4 - A6  Column loop with error compensation and lazy block updates.
+ *
+ * For each column i in natural order (FDE breakdown figure steps 1-4): q_i = clamp(rint(w_i/scale)
+ * + zero, 0, 2^b-1); err = (w_i - scale*(q_i - zero)) / U_ii; W[:, j] -= err * U[i, j] for the
+ * remaining columns j of the block at once, and for the columns after the block once per block.
+ * Grid: asymmetric min/max over the row (per-row, from the original W) or over the group's current
+ * values when the loop reaches the group (per-group), the range widened to contain 0.  The grid
+ * decisions (zero point and codes) use IEEE fp32 division and round-half-to-even.
+ *
+ *   W          [m, d] row-major, dtype w_dtype (FP16, BF16 or FP32); read only.
+ *   U          [d, d] fp32 upper factor from gptq_prepare_uinv (strict lower part ignored).
+ *   codes      [m, d] uint8 output, one code per weight.
+ *   scales     [m, n_groups] fp32 output, n_groups = group_size ? d / group_size : 1.
+ *   zeros      [m, n_groups] int32 output.
+ *   workspace  >= gptq_quantize_workspace_size(m, d, cfg) bytes, 256-byte aligned (holds the
+ *              working copy of W in fp32 and the per-block errors).
+ *   Requires d % 32 == 0 and d % block_size == 0.  flags & GPTQ_FLAG_ACT_ORDER -> UNSUPPORTED.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_quantize_layer(const void* W, int32_t w_dtype, int64_t m, int64_t d,
+                                const float* U, const gptq_quant_cfg* cfg, uint8_t* codes,
+                                float* scales, int32_t* zeros, void* workspace,
+                                size_t workspace_bytes, void* stream);
+GPTQ_API size_t gptq_quantize_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* cfg);
+
+/* ------------------------------------------------------------------------------------------
+ * A7  Pack b-bit codes into int32 words (storage of 3-/4-bit weights for the inference kernel;
+ * FDE breakdown figure, "3-bit weights 66 GB").  Layout: per row a little-endian bit stream, code j
+ * in bits [j*b, (j+1)*b), word k = stream bits [32k, 32k+32).  Row stride = d*bits/32 words.
+ *
+ *   codes      [m, d] uint8, each < 2^bits (higher bits are masked off).
+ *   packed     [m, d*bits/32] int32 output.  Requires d % 32 == 0, bits in {2, 3, 4}.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_pack(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,
+                      void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Status helpers.
+ * gptq_read_status: synchronizes `stream`, copies the device status word to the host, returns the
+ * code it holds (GPTQ_OK if clear) and stores its detail (e.g. the failing pivot) in *detail when
+ * detail is not NULL.  Returns GPTQ_ERR_CUDA if the copy fails.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_read_status(const int32_t* dev_status, void* stream, int64_t* detail);
+GPTQ_API const char* gptq_status_string(int32_t status);
+GPTQ_API int32_t gptq_abi_version(void);
+
+/* Diagnostics: total number of CUDA kernels this library has launched in the process (all devices,
+ * all threads).  Host-side counter; reading it does not touch the device. */
+GPTQ_API uint64_t gptq_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTQ_B200_H */

@@ -1,0 +1,242 @@
+"""GPTQ layer-wise quantization solver for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libgptq.so`` (C ABI in ``include/gptq.h``).  The functions keep the C
+names and only marshal arguments: torch tensors supply device memory and streams, and every step of
+the solver runs in the library's CUDA kernels.  There is no CPU fallback; if the library is missing,
+the first call raises.
+
+    H = 2 X^T X                       gptq_hessian_accumulate
+    U = chol((H + l*mean(diag H) I)^-1) gptq_prepare_uinv
+    codes, scales, zeros              gptq_quantize_layer   (column loop + lazy block updates)
+    packed int32 words                gptq_pack
+
+``LayerSolver`` strings the four calls together over preallocated buffers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "GPTQError", "lib", "gptq_hessian_accumulate", "gptq_hessian_workspace_size", "gptq_prepare_uinv",
+    "gptq_prepare_workspace_size", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
+    "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
+
+GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_UNSUPPORTED, GPTQ_ERR_NOT_PD = 0, 1, 2, 3
+GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
+GPTQ_BF16, GPTQ_FP16, GPTQ_FP32 = 0, 1, 2
+GPTQ_FLAG_ACT_ORDER = 1
+
+_DTYPES = {torch.bfloat16: GPTQ_BF16, torch.float16: GPTQ_FP16, torch.float32: GPTQ_FP32}
+
+
+class QuantCfg(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+_i32, _i64, _sz, _vp, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+ABI_FUNCTIONS = {
+    "gptq_hessian_accumulate": (_i32, [_vp, _i32, _i64, _i64, _vp, _f32, _i32, _vp, _vp, _sz, _vp]),
+    "gptq_hessian_workspace_size": (_sz, [_i64, _i64, _i32]),
+    "gptq_prepare_uinv": (_i32, [_vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "gptq_prepare_workspace_size": (_sz, [_i64]),
+    "gptq_quantize_layer": (_i32, [_vp, _i32, _i64, _i64, _vp, ctypes.POINTER(QuantCfg), _vp, _vp, _vp,
+                                   _vp, _sz, _vp]),
+    "gptq_quantize_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
+    "gptq_pack": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp]),
+    "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
+    "gptq_status_string": (ctypes.c_char_p, [_i32]),
+    "gptq_abi_version": (_i32, []),
+    "gptq_kernel_launches": (ctypes.c_uint64, []),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library (loaded on first use; raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m post_weight_quantization_21_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in ABI_FUNCTIONS.items():
+            fn = getattr(handle, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = handle
+    return _lib
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: int | None = None):
+        self.status, self.detail = status, detail
+        msg = f"{where}: {gptq_status_string(status)} (status {status})"
+        if detail is not None:
+            msg += f", detail {detail}"
+        super().__init__(msg)
+
+
+def gptq_status_string(status: int) -> str:
+    return lib().gptq_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != GPTQ_OK:
+        raise GPTQError(status, where)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _cfg(bits: int, group_size: int, block_size: int, flags: int = 0) -> QuantCfg:
+    return QuantCfg(bits, group_size, block_size, flags)
+
+
+def _contig(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+# ------------------------------------------------------------------------------------------ A1
+def gptq_hessian_workspace_size(n_tokens: int, d: int, x_dtype: torch.dtype) -> int:
+    return lib().gptq_hessian_workspace_size(n_tokens, d, _DTYPES[x_dtype])
+
+
+def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, status: torch.Tensor, workspace: torch.Tensor,
+                            scale: float = 2.0, accumulate: bool = False, stream=None):
+    """H (upper triangle) = [H +] scale * X^T X for X [tokens, d] on the device."""
+    _contig(X, "X"), _contig(H, "H")
+    n, d = X.shape
+    st = lib().gptq_hessian_accumulate(_ptr(X), _DTYPES[X.dtype], n, d, _ptr(H), scale, int(accumulate),
+                                       _ptr(status), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream))
+    _check(st, "gptq_hessian_accumulate")
+
+
+# ------------------------------------------------------------------------------------------ A2 + A3
+def gptq_prepare_workspace_size(d: int) -> int:
+    return lib().gptq_prepare_workspace_size(d)
+
+
+def gptq_prepare_uinv(H: torch.Tensor, U: torch.Tensor, status: torch.Tensor, workspace: torch.Tensor,
+                      damp: float = 0.01, stream=None):
+    """U = upper Cholesky factor of (H + damp*mean(diag H)*I)^-1 (device status in ``status``)."""
+    _contig(H, "H"), _contig(U, "U")
+    st = lib().gptq_prepare_uinv(_ptr(H), H.shape[0], damp, _ptr(U), _ptr(status), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "gptq_prepare_uinv")
+
+
+# ------------------------------------------------------------------------------------------ A4 - A6
+def gptq_quantize_workspace_size(m: int, d: int, bits: int, group_size: int, block_size: int) -> int:
+    c = _cfg(bits, group_size, block_size)
+    return lib().gptq_quantize_workspace_size(m, d, ctypes.byref(c))
+
+
+def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                        zeros: torch.Tensor, workspace: torch.Tensor, bits: int, group_size: int = 0,
+                        block_size: int = 128, flags: int = 0, stream=None):
+    """Column loop with lazy block updates: fills codes [m, d] u8, scales/zeros [m, n_groups]."""
+    for t, n in ((W, "W"), (U, "U"), (codes, "codes"), (scales, "scales"), (zeros, "zeros")):
+        _contig(t, n)
+    m, d = W.shape
+    c = _cfg(bits, group_size, block_size, flags)
+    st = lib().gptq_quantize_layer(_ptr(W), _DTYPES[W.dtype], m, d, _ptr(U), ctypes.byref(c), _ptr(codes),
+                                   _ptr(scales), _ptr(zeros), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "gptq_quantize_layer")
+
+
+# ------------------------------------------------------------------------------------------ A7
+def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None):
+    _contig(codes, "codes"), _contig(packed, "packed")
+    m, d = codes.shape
+    _check(lib().gptq_pack(_ptr(codes), m, d, bits, _ptr(packed), _stream(stream)), "gptq_pack")
+
+
+def gptq_kernel_launches() -> int:
+    """Kernels launched by the library so far in this process (host-side counter)."""
+    return int(lib().gptq_kernel_launches())
+
+
+def gptq_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:
+    detail = ctypes.c_int64(0)
+    code = lib().gptq_read_status(_ptr(status), _stream(stream), ctypes.byref(detail))
+    return int(code), int(detail.value)
+
+
+# ------------------------------------------------------------------------------------------ solver
+class LayerSolver:
+    """Device buffers for one layer shape, and the four calls in order.
+
+    ``run()`` works on the device-resident ``X``/``W`` buffers; ``run_host()`` copies pinned host
+    inputs in, runs, and copies the packed codes, scales and zeros back out.
+    """
+
+    def __init__(self, m: int, d: int, n_tokens: int, bits: int, group_size: int = 0, block_size: int = 128,
+                 damp: float = 0.01, x_dtype=torch.bfloat16, w_dtype=torch.float16, device="cuda"):
+        self.m, self.d, self.n_tokens = m, d, n_tokens
+        self.bits, self.group_size, self.block_size, self.damp = bits, group_size, block_size, damp
+        n_groups = 1 if group_size == 0 else d // group_size
+        dev = torch.device(device)
+        u8 = torch.uint8
+        self.X = torch.empty(n_tokens, d, dtype=x_dtype, device=dev)
+        self.W = torch.empty(m, d, dtype=w_dtype, device=dev)
+        self.H = torch.empty(d, d, dtype=torch.float32, device=dev)
+        self.U = torch.empty(d, d, dtype=torch.float32, device=dev)
+        self.codes = torch.empty(m, d, dtype=u8, device=dev)
+        self.scales = torch.empty(m, n_groups, dtype=torch.float32, device=dev)
+        self.zeros = torch.empty(m, n_groups, dtype=torch.int32, device=dev)
+        self.packed = torch.empty(m, d * bits // 32, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        ws = max(gptq_hessian_workspace_size(n_tokens, d, x_dtype), gptq_prepare_workspace_size(d),
+                 gptq_quantize_workspace_size(m, d, bits, group_size, block_size), 256)
+        self.workspace = torch.empty(ws, dtype=u8, device=dev)
+
+    def hessian(self, stream=None):
+        gptq_hessian_accumulate(self.X, self.H, self.status, self.workspace, 2.0, False, stream)
+
+    def prepare(self, stream=None):
+        gptq_prepare_uinv(self.H, self.U, self.status, self.workspace, self.damp, stream)
+
+    def quantize(self, stream=None):
+        gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.workspace, self.bits,
+                            self.group_size, self.block_size, 0, stream)
+
+    def pack(self, stream=None):
+        gptq_pack(self.codes, self.bits, self.packed, stream)
+
+    def run(self, stream=None):
+        self.hessian(stream)
+        self.prepare(stream)
+        self.quantize(stream)
+        self.pack(stream)
+
+    def check_status(self, stream=None):
+        code, detail = gptq_read_status(self.status, stream)
+        if code != GPTQ_OK:
+            raise GPTQError(code, "device status", detail)
+
+    def run_host(self, W_host: torch.Tensor, X_host: torch.Tensor, out_packed: torch.Tensor,
+                 out_scales: torch.Tensor, out_zeros: torch.Tensor, stream=None):
+        """Host -> device copies of W and X, the four calls, device -> host copies of the results."""
+        self.X.copy_(X_host, non_blocking=True)
+        self.W.copy_(W_host, non_blocking=True)
+        self.run(stream)
+        out_packed.copy_(self.packed, non_blocking=True)
+        out_scales.copy_(self.scales, non_blocking=True)
+        out_zeros.copy_(self.zeros, non_blocking=True)

@@ -1,0 +1,75 @@
+// Shared helpers of the GPTQ solver kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gptq.h"
+
+#define GPTQ_CUDA_TRY(expr)                                  \
+  do {                                                       \
+    cudaError_t e__ = (expr);                                \
+    if (e__ != cudaSuccess) return GPTQ_ERR_CUDA;            \
+  } while (0)
+
+namespace gptq {
+void count_launch();
+}
+// Called right after every kernel launch: counts it and reports a failed launch.
+#define GPTQ_LAUNCH_CHECK()      \
+  do {                           \
+    gptq::count_launch();        \
+    GPTQ_CUDA_TRY(cudaGetLastError()); \
+  } while (0)
+
+namespace gptq {
+
+constexpr int kWarp = 32;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Records the first device-side failure in the caller's status word {code, detail}.
+__device__ __forceinline__ void report_status(int32_t* status, int32_t code, int32_t detail) {
+  if (status == nullptr) return;
+  if (atomicCAS(status, 0, code) == 0) status[1] = detail;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Asymmetric min/max grid: the range widened to contain 0, an empty range becomes [-1, 1];
+// scale = (hi - lo) / maxq and zero = rint(-lo / scale), both in IEEE fp32.
+__device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, float& scale,
+                                                float& zero) {
+  float lo = fminf(mn, 0.0f);
+  float hi = fmaxf(mx, 0.0f);
+  if (lo == hi) {
+    lo = -1.0f;
+    hi = 1.0f;
+  }
+  scale = __fdiv_rn(hi - lo, maxq);
+  zero = rintf(__fdiv_rn(-lo, scale));
+}
+
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+}  // namespace gptq

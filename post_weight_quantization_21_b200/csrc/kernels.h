@@ -1,0 +1,40 @@
+// Internal launchers of the GPTQ solver kernels (host side; not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gptq.h"
+
+namespace gptq {
+
+// A1, fp32 FMA path (any input dtype; the product path for fp32 inputs)
+size_t hessian_simt_workspace(int64_t n_tokens, int64_t d);
+gptq_status hessian_simt_launch(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d, float* H,
+                                float scale, int32_t accumulate, void* workspace, cudaStream_t stream);
+
+// A2 + A3
+size_t prepare_workspace(int64_t d);
+gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
+                           void* workspace, cudaStream_t stream);
+
+// A4 - A6
+size_t quantize_workspace(int64_t m, int64_t d, int block_size);
+gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U,
+                            const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
+                            void* workspace, cudaStream_t stream);
+
+// A7
+gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,
+                        cudaStream_t stream);
+
+}  // namespace gptq
+
+namespace gptq {
+// A1 dispatcher: tensor cores for 16-bit inputs, fp32 FMA for fp32 inputs.
+size_t hessian_workspace(int64_t n_tokens, int64_t d, int32_t x_dtype);
+gptq_status hessian_launch(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d, float* H,
+                           float scale, int32_t accumulate, int32_t* status, void* workspace,
+                           cudaStream_t stream);
+}  // namespace gptq

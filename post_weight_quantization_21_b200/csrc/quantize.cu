@@ -1,0 +1,271 @@
+// A4 - A7: grid, column loop with error compensation, lazy block updates, packing.
+//
+// GPTQ's column loop (FDE Interviews breakdown of GPTQ, figure "THE IDEA, VISUALLY"):
+//   1. round column i to the b-bit grid;  2. err = (w_i - q_i) / U_ii;
+//   3. W[:, i+1:] -= err * U[i, i+1:];   4. apply in blocks of 128 columns.
+// Rows are independent once U is known (section 01: one column order shared by every row), so a
+// warp owns a row: lane l holds columns l, l+32, l+64, l+96 of the current block in registers and
+// the block's 128x128 corner of U sits in shared memory.  Each step broadcasts w_i with one
+// shuffle, rounds it, and updates the four register columns; the block never leaves the SM.
+// Step 4 is a separate tiled fp32 GEMM per block: W[:, i2:] -= Err[:, i1:i2] U[i1:i2, i2:].
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gptq {
+namespace {
+
+constexpr int kRowsPerCta = 8;  // one warp per row
+
+// w_work = float(W); per-row grid from the original row when group_size == 0.
+template <typename T>
+__global__ void __launch_bounds__(256) convert_rowgrid_kernel(const T* __restrict__ W, int64_t m, int d,
+                                                              int bits, int group_size,
+                                                              float* __restrict__ w_work,
+                                                              float* __restrict__ scales,
+                                                              int32_t* __restrict__ zeros) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
+  if (row >= m) return;
+  const T* src = W + row * d;
+  float* dst = w_work + row * d;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int c = lane; c < d; c += 32) {
+    const float v = to_f32(src[c]);
+    dst[c] = v;
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  if (group_size == 0) {
+    mn = warp_min(mn);
+    mx = warp_max(mx);
+    if (lane == 0) {
+      float s, z;
+      grid_from_range(mn, mx, (float)((1 << bits) - 1), s, z);
+      scales[row] = s;
+      zeros[row] = (int32_t)z;
+    }
+  }
+}
+
+// Column loop over block [i1, i1 + 32*NS) for 8 rows per CTA.
+template <int NS>
+__global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
+                                                      const float* __restrict__ U, int bits,
+                                                      int group_size, uint8_t* __restrict__ codes,
+                                                      float* __restrict__ scales,
+                                                      int32_t* __restrict__ zeros,
+                                                      float* __restrict__ err_out) {
+  constexpr int B = 32 * NS;
+  extern __shared__ float sm[];
+  float* Us = sm;           // [B][B], strict lower part zero
+  float* invd = sm + B * B;  // [B]
+  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
+    const int r = e / B, c = e % B;
+    Us[e] = (c > r) ? U[(size_t)(i1 + r) * d + i1 + c] : 0.0f;
+  }
+  for (int r = threadIdx.x; r < B; r += blockDim.x) invd[r] = 1.0f / U[(size_t)(i1 + r) * d + i1 + r];
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
+  if (row >= m) return;
+  float* wr = w + row * d;
+  float v[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) v[s] = wr[i1 + s * 32 + lane];
+  const float maxq = (float)((1 << bits) - 1);
+  const int n_groups = group_size ? d / group_size : 1;
+  float scale = 0.f, zero = 0.f;
+  if (group_size == 0) {
+    scale = scales[row];
+    zero = (float)zeros[row];
+  } else if (i1 % group_size != 0) {  // block inside a group that started in an earlier block
+    scale = scales[row * n_groups + i1 / group_size];
+    zero = (float)zeros[row * n_groups + i1 / group_size];
+  }
+  uint32_t code_reg[NS];
+  float err_reg[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+#pragma unroll
+    for (int l = 0; l < 32; ++l) {
+      const int i = s * 32 + l;
+      if (l == 0 && group_size != 0 && ((i1 + i) % group_size) == 0) {
+        // grid of the group starting here, from the current values of its columns
+        const int gw = group_size / 32;  // slots covered inside the block
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < NS; ++t)
+          if (t >= s && t < s + gw) {
+            mn = fminf(mn, v[t]);
+            mx = fmaxf(mx, v[t]);
+          }
+        for (int c = i1 + B + lane; c < i1 + i + group_size; c += 32) {  // group wider than block
+          const float x = wr[c];
+          mn = fminf(mn, x);
+          mx = fmaxf(mx, x);
+        }
+        mn = warp_min(mn);
+        mx = warp_max(mx);
+        grid_from_range(mn, mx, maxq, scale, zero);
+        if (lane == 0) {
+          const int g = (i1 + i) / group_size;
+          scales[row * n_groups + g] = scale;
+          zeros[row * n_groups + g] = (int32_t)zero;
+        }
+      }
+      const float wi = __shfl_sync(0xffffffffu, v[s], l);
+      float q = rintf(__fdiv_rn(wi, scale)) + zero;
+      q = fminf(fmaxf(q, 0.0f), maxq);
+      const float deq = scale * (q - zero);
+      const float err = (wi - deq) * invd[i];
+      if (lane == l) {
+        code_reg[s] = (uint32_t)q;
+        err_reg[s] = err;
+      }
+      const float* urow = Us + i * B;
+#pragma unroll
+      for (int t = 0; t < NS; ++t) v[t] = fmaf(-err, urow[t * 32 + lane], v[t]);
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    codes[row * d + i1 + s * 32 + lane] = (uint8_t)code_reg[s];
+    err_out[row * B + s * 32 + lane] = err_reg[s];
+  }
+}
+
+// w[:, i2:] -= Err[:, 0:B] * U[i1:i1+B, i2:]; 64x64 output tile per CTA, K = B in steps of 32.
+template <int B>
+__global__ void __launch_bounds__(256) lazy_update_kernel(float* __restrict__ w, int64_t m, int d, int i1,
+                                                          const float* __restrict__ U,
+                                                          const float* __restrict__ err) {
+  constexpr int KC = 32;
+  __shared__ __align__(16) float Et[KC][64 + 4];  // Et[k][row]
+  __shared__ __align__(16) float Ut[KC][64 + 4];  // Ut[k][col]
+  const int i2 = i1 + B;
+  const int64_t r0 = (int64_t)blockIdx.x * 64;  // row tiles on x (up to 2^31 - 1)
+  const int c0 = i2 + blockIdx.y * 64;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < B; k0 += KC) {
+    for (int e = threadIdx.x; e < 64 * KC; e += blockDim.x) {
+      const int r = e / KC, k = e % KC;
+      const int64_t gr = r0 + r;
+      Et[k][r] = (gr < m) ? err[gr * B + k0 + k] : 0.0f;
+    }
+    for (int e = threadIdx.x; e < 64 * KC; e += blockDim.x) {
+      const int k = e / 64, c = e % 64;
+      Ut[k][c] = (c0 + c < d) ? U[(size_t)(i1 + k0 + k) * d + c0 + c] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < KC; ++k) {
+      const float4 a = *reinterpret_cast<const float4*>(&Et[k][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Ut[k][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int64_t gr = r0 + ty * 4 + p;
+    if (gr >= m) continue;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int gc = c0 + tx * 4 + q;
+      if (gc < d) w[gr * d + gc] -= acc[p][q];
+    }
+  }
+}
+
+// One thread per int32 word of the packed row stream.
+__global__ void pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int d, int bits,
+                            int32_t* __restrict__ packed) {
+  const int wpr = d * bits / 32;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= m * wpr) return;
+  const int64_t row = idx / wpr;
+  const int k = (int)(idx % wpr);
+  const uint32_t mask = (1u << bits) - 1u;
+  const int bit0 = 32 * k;
+  const int j0 = bit0 / bits, j1 = (bit0 + 31) / bits;
+  const uint8_t* cr = codes + row * d;
+  uint32_t word = 0;
+  for (int j = j0; j <= j1 && j < d; ++j) {
+    const uint32_t c = (uint32_t)cr[j] & mask;
+    const int sh = j * bits - bit0;
+    word |= (sh >= 0) ? (c << sh) : (c >> (-sh));
+  }
+  packed[idx] = (int32_t)word;
+}
+
+template <typename T>
+void launch_convert(const void* W, int64_t m, int d, int bits, int gs, float* ww, float* sc, int32_t* z,
+                    cudaStream_t s) {
+  const int grid = (int)((m + kRowsPerCta - 1) / kRowsPerCta);
+  convert_rowgrid_kernel<T><<<grid, 256, 0, s>>>(static_cast<const T*>(W), m, d, bits, gs, ww, sc, z);
+}
+
+template <int NS>
+gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, int gs, uint8_t* codes,
+                       float* scales, int32_t* zeros, float* err, cudaStream_t s) {
+  constexpr int B = 32 * NS;
+  const int smem = (B * B + B) * sizeof(float);
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int grid_rows = (int)((m + kRowsPerCta - 1) / kRowsPerCta);
+  for (int i1 = 0; i1 < d; i1 += B) {
+    colloop_kernel<NS><<<grid_rows, 256, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
+    GPTQ_LAUNCH_CHECK();
+    const int rest = d - (i1 + B);
+    if (rest > 0) {
+      dim3 grid((unsigned)((m + 63) / 64), (rest + 63) / 64);
+      lazy_update_kernel<B><<<grid, 256, 0, s>>>(ww, m, d, i1, U, err);
+      GPTQ_LAUNCH_CHECK();
+    }
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+size_t quantize_workspace(int64_t m, int64_t d, int block_size) {
+  return align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * block_size * sizeof(float), 256);
+}
+
+gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d64, const float* U,
+                            const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
+                            void* workspace, cudaStream_t s) {
+  const int d = (int)d64;
+  char* ws = static_cast<char*>(workspace);
+  float* ww = reinterpret_cast<float*>(ws);
+  float* err = reinterpret_cast<float*>(ws + align_up((size_t)m * d * sizeof(float), 256));
+  switch (w_dtype) {
+    case GPTQ_FP32: launch_convert<float>(W, m, d, cfg.bits, cfg.group_size, ww, scales, zeros, s); break;
+    case GPTQ_FP16: launch_convert<__half>(W, m, d, cfg.bits, cfg.group_size, ww, scales, zeros, s); break;
+    case GPTQ_BF16: launch_convert<__nv_bfloat16>(W, m, d, cfg.bits, cfg.group_size, ww, scales, zeros, s); break;
+    default: return GPTQ_ERR_ARG;
+  }
+  GPTQ_LAUNCH_CHECK();
+  switch (cfg.block_size) {
+    case 32: return run_blocks<1>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, s);
+    case 64: return run_blocks<2>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, s);
+    case 128: return run_blocks<4>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, s);
+    default: return GPTQ_ERR_ARG;
+  }
+}
+
+gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,
+                        cudaStream_t s) {
+  const int64_t n = m * (d * bits / 32);
+  if (n == 0) return GPTQ_OK;
+  const int threads = 256;
+  pack_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(codes, m, (int)d, bits, packed);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -1,0 +1,81 @@
+"""The C-ABI library: it loads, exports every entry point include/gptq.h declares, and its host-side
+validation rejects bad arguments before any device work (no GPU needed for these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import post_weight_quantization_21_b200 as g
+from post_weight_quantization_21_b200 import build as gbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gptq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(g.LIB_PATH):
+        gbuild.build()
+    return g.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"GPTQ_API\s+[\w\s\*]+?\b(gptq_\w+)\s*\(", src)
+
+
+def test_header_declares_the_four_calls():
+    names = set(declared_functions())
+    for n in ("gptq_hessian_accumulate", "gptq_prepare_uinv", "gptq_quantize_layer", "gptq_pack"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(g.ABI_FUNCTIONS)
+    assert lib.gptq_abi_version() == 1
+
+
+def test_status_strings(lib):
+    assert g.gptq_status_string(0) == "ok"
+    assert "positive definite" in g.gptq_status_string(3)
+
+
+def test_workspace_sizes(lib):
+    import torch
+    assert g.gptq_hessian_workspace_size(262144, 768, torch.bfloat16) > 0
+    assert g.gptq_prepare_workspace_size(4096) >= 4096 * 64 * 4
+    w = g.gptq_quantize_workspace_size(64, 128, 4, 0, 32)
+    assert w >= 64 * 128 * 4 + 64 * 32 * 4
+    assert g.gptq_quantize_workspace_size(64, 128, 5, 0, 32) == 0       # bits out of range
+    assert g.gptq_quantize_workspace_size(64, 100, 4, 0, 32) == 0       # block does not divide d
+    assert lib.gptq_prepare_workspace_size(0) == 0
+
+
+def test_validation_rejects_bad_arguments_without_a_device(lib):
+    cfg = g.QuantCfg(4, 0, 128, 0)
+    fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    st = lib.gptq_quantize_layer(fake, 1, 8, 100, fake, ctypes.byref(cfg), fake, fake, fake, fake, 1 << 20, None)
+    assert st == g.GPTQ_ERR_ARG                               # d % 32 != 0
+    bad = g.QuantCfg(5, 0, 128, 0)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(bad), fake, fake, fake, fake, 1 << 20, None)
+    assert st == g.GPTQ_ERR_ARG                               # bits = 5
+    act = g.QuantCfg(4, 0, 128, g.GPTQ_FLAG_ACT_ORDER)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(act), fake, fake, fake, fake, 1 << 20, None)
+    assert st == g.GPTQ_ERR_UNSUPPORTED
+    grp = g.QuantCfg(4, 96, 128, 0)                           # 96 and 128 do not divide one another
+    st = lib.gptq_quantize_layer(fake, 1, 8, 384, fake, ctypes.byref(grp), fake, fake, fake, fake, 1 << 20, None)
+    assert st == g.GPTQ_ERR_ARG
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(cfg), fake, fake, fake, None, 0, None)
+    assert st == g.GPTQ_ERR_WORKSPACE
+    assert lib.gptq_pack(fake, 4, 48, 3, fake, None) == g.GPTQ_ERR_ARG        # d % 32
+    assert lib.gptq_pack(fake, 4, 64, 5, fake, None) == g.GPTQ_ERR_ARG        # bits
+    assert lib.gptq_hessian_accumulate(fake, 0, 16, 12, fake, 2.0, 0, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG
+    assert lib.gptq_hessian_accumulate(fake, 7, 16, 16, fake, 2.0, 0, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG
+    other = ctypes.c_void_p(4096)
+    assert lib.gptq_prepare_uinv(fake, 16, 0.01, other, fake, None, 0, None) == g.GPTQ_ERR_WORKSPACE
+    assert lib.gptq_prepare_uinv(fake, 16, -1.0, other, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG
+    assert lib.gptq_prepare_uinv(fake, 16, 0.01, fake, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG  # H == U

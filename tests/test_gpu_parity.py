@@ -1,0 +1,172 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle on the same seeded inputs.
+
+Each test calls the library through its C ABI (ctypes binding) and compares element by element with
+the oracle at sizes the oracle finishes in seconds (several tiles and a ragged tail), plus the
+bench's full-size layer (opt125m 768x768, 262,144 tokens) end to end.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_21_b200 import workloads as wl
+
+import gpu_support as S
+
+pytestmark = pytest.mark.gpu
+
+
+def _x(n, d, dtype, seed, corr=True):
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn(n, d, generator=gen, dtype=torch.float64)
+    if corr:
+        A = torch.randn(d, d, generator=gen, dtype=torch.float64) / d ** 0.5
+        x = x @ A + 0.3 * torch.randn(n, d, generator=gen, dtype=torch.float64)
+    return x.to(dtype)
+
+
+# ------------------------------------------------------------------------------------------ A1
+@pytest.mark.parametrize("n,d,dtype", [
+    (256, 128, torch.float32),       # the tiny layer
+    (1000, 200, torch.float32),      # ragged tile tail, ragged token tail
+    (5000, 200, torch.bfloat16),
+    (3000, 136, torch.float16),
+    (2048 * 9 + 17, 520, torch.bfloat16),
+])
+def test_hessian_matches_oracle(n, d, dtype):
+    X = _x(n, d, dtype, seed=n + d)
+    H = S.hessian(X.to(S.dev())).cpu().numpy()
+    Href = oracle.hessian(X.double().numpy())
+    assert S.upper_rel_fro(H, Href) <= S.H_REL_FRO
+
+
+def test_hessian_accumulates_and_handles_empty_input():
+    X = _x(4096, 64, torch.bfloat16, seed=5).to(S.dev())
+    H = S.hessian(X[:1000])
+    S.hessian(X[1000:], accumulate_into=H)
+    Href = oracle.hessian(X.cpu().double().numpy())
+    assert S.upper_rel_fro(H.cpu().numpy(), Href) <= S.H_REL_FRO
+    H0 = S.hessian(X[:0])                          # 0 tokens, overwrite mode: H = 0
+    assert torch.count_nonzero(torch.triu(H0)) == 0
+    S.hessian(X[:0], accumulate_into=H)            # 0 tokens, accumulate mode: unchanged
+    assert S.upper_rel_fro(H.cpu().numpy(), Href) <= S.H_REL_FRO
+
+
+def test_hessian_full_size_opt125m_layer():
+    L = wl.LAYERS["opt125m_768x768"]
+    X = wl.make_x(L)
+    H = S.hessian(X.to(S.dev())).cpu().numpy()
+    Href = oracle.hessian(X.double().numpy())
+    assert S.upper_rel_fro(H, Href) <= S.H_REL_FRO
+
+
+# ------------------------------------------------------------------------------------------ A2 + A3
+@pytest.mark.parametrize("d", [1, 5, 64, 128, 200, 768, 1000])
+def test_prepare_matches_oracle(d):
+    n = max(4 * d, 64)
+    X = _x(n, d, torch.float64, seed=d)
+    H = oracle.hessian(X.numpy())
+    Hd = oracle.dampen(H, 0.01)
+    Uref = oracle.inverse_upper_cholesky(Hd)
+    U = S.prepare(torch.from_numpy(H).float().to(S.dev())).cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(U, -1) == 0.0)
+    rel = np.linalg.norm(U - Uref) / np.linalg.norm(Uref)
+    res = np.linalg.norm(U @ Hd @ U.T - np.eye(d)) / np.sqrt(d)
+    kappa = np.linalg.cond(Hd)
+    # fp32 factorisation: forward error ~ kappa * eps32; residual ~ d * eps32
+    assert rel <= max(1e-5, 10 * kappa * 6e-8), (rel, kappa)
+    assert res <= 1e-4, res
+
+
+def test_prepare_reports_indefinite_matrix():
+    d = 96
+    H = torch.eye(d) * 2.0
+    H[37, 37] = -50.0  # damping 0.01 * mean(diag) cannot lift this pivot
+    U, code, detail = S.prepare(H.to(S.dev()), expect_ok=False)
+    assert code == 3  # GPTQ_ERR_NOT_PD
+    assert detail == 37
+
+
+# ------------------------------------------------------------------------------------------ A4 - A6
+QUANT_CASES = [
+    # m, d, bits, group, block
+    (64, 128, 4, 0, 32),
+    (100, 256, 3, 0, 128),
+    (37, 512, 2, 0, 64),
+    (64, 512, 3, 128, 128),
+    (64, 512, 4, 32, 128),
+    (64, 512, 4, 256, 128),
+    (48, 384, 4, 64, 32),
+    (1, 128, 4, 0, 128),
+]
+
+
+@pytest.mark.parametrize("m,d,bits,gs,B", QUANT_CASES)
+def test_quantize_matches_oracle_given_U(m, d, bits, gs, B):
+    X = _x(4 * d, d, torch.float64, seed=m * d + bits)
+    H = oracle.hessian(X.numpy())
+    U = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01))
+    U32 = U.astype(np.float32)
+    W = (torch.randn(m, d, generator=torch.Generator().manual_seed(d + m)) * 0.02).half()
+    ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), bits, gs, B)
+    gpu = S.quantize(W.to(S.dev()), torch.from_numpy(U32).to(S.dev()), bits, gs, B)
+    S.compare_quantization(gpu, ref, gs, W.double().numpy(), H, label=f"{m}x{d} b{bits} g{gs} B{B}")
+
+
+def test_quantize_fp32_and_bf16_weights():
+    d, m = 256, 32
+    X = _x(4 * d, d, torch.float64, seed=3)
+    H = oracle.hessian(X.numpy())
+    U32 = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01)).astype(np.float32)
+    for dt in (torch.float32, torch.bfloat16):
+        W = (torch.randn(m, d, generator=torch.Generator().manual_seed(1)) * 0.02).to(dt)
+        ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), 4, 0, 128)
+        gpu = S.quantize(W.to(S.dev()), torch.from_numpy(U32).to(S.dev()), 4, 0, 128)
+        S.compare_quantization(gpu, ref, 0, W.double().numpy(), H, label=str(dt))
+
+
+# ------------------------------------------------------------------------------------------ A7
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("m,d", [(1, 32), (7, 96), (33, 768)])
+def test_pack_bit_exact(bits, m, d):
+    codes = torch.randint(0, 2 ** bits, (m, d), generator=torch.Generator().manual_seed(m + d + bits),
+                          dtype=torch.uint8)
+    got = S.pack(codes.to(S.dev()), bits)
+    np.testing.assert_array_equal(got, oracle.pack_codes(codes.numpy().astype(np.int64), bits))
+
+
+# ------------------------------------------------------------------------------------------ end to end
+def _layer_end_to_end(L, check_h=True):
+    W = wl.make_w(L)
+    X = wl.make_x(L)
+    from post_weight_quantization_21_b200 import LayerSolver
+    s = LayerSolver(L.m, L.d, L.n_tokens, L.bits, L.group_size, L.block_size, L.damp, X.dtype, W.dtype)
+    s.X.copy_(X)
+    s.W.copy_(W)
+    s.run()
+    s.check_status()
+    torch.cuda.synchronize()
+    ref = oracle.gptq_layer(W.double().numpy(), X.double().numpy(), L.bits, L.group_size, L.block_size, L.damp)
+    if check_h:
+        assert S.upper_rel_fro(s.H.cpu().numpy(), ref["H"]) <= S.H_REL_FRO
+    gpu = (s.codes.cpu().numpy().astype(np.int64), s.scales.cpu().numpy(), s.zeros.cpu().numpy().astype(np.int64))
+    stats = S.compare_quantization(gpu, ref, L.group_size, W.double().numpy(), ref["H"], ref["E"], label=L.name)
+    np.testing.assert_array_equal(s.packed.cpu().numpy(), oracle.pack_codes(gpu[0], L.bits))
+    return stats
+
+
+def test_end_to_end_tiny_layer():
+    _layer_end_to_end(wl.LAYERS["tiny_64x128"])
+
+
+def test_end_to_end_opt125m_layer():
+    st = _layer_end_to_end(wl.LAYERS["opt125m_768x768"])
+    print("opt125m end-to-end", st)
+
+
+def test_end_to_end_reduced_llama_q_layer():
+    """The 3-bit group-128 setting on a 1024-wide slice of the q_proj layer (all stages chained)."""
+    L = wl.LAYERS["llama7b_q_4096x4096"]
+    import dataclasses
+    L = dataclasses.replace(L, m=512, d=1024, n_tokens=16 * 2048)
+    _layer_end_to_end(L)
