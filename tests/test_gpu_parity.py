@@ -106,7 +106,7 @@ def test_quantize_matches_oracle_given_U(m, d, bits, gs, B):
     X = _x(4 * d, d, torch.float64, seed=m * d + bits)
     H = oracle.hessian(X.numpy())
     U = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01))
-    U32 = U.astype(np.float32)
+    U32 = np.ascontiguousarray(U, dtype=np.float32)
     W = (torch.randn(m, d, generator=torch.Generator().manual_seed(d + m)) * 0.02).half()
     ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), bits, gs, B)
     gpu = S.quantize(W.to(S.dev()), torch.from_numpy(U32).to(S.dev()), bits, gs, B)
@@ -117,7 +117,7 @@ def test_quantize_fp32_and_bf16_weights():
     d, m = 256, 32
     X = _x(4 * d, d, torch.float64, seed=3)
     H = oracle.hessian(X.numpy())
-    U32 = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01)).astype(np.float32)
+    U32 = np.ascontiguousarray(oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01)), dtype=np.float32)
     for dt in (torch.float32, torch.bfloat16):
         W = (torch.randn(m, d, generator=torch.Generator().manual_seed(1)) * 0.02).to(dt)
         ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), 4, 0, 128)
