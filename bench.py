@@ -341,7 +341,7 @@ def main():
 
 
 def hessian_sources():
-    return ["post_weight_quantization_21_b200/csrc/hessian.cu", "post_weight_quantization_21_b200/csrc/hessian_simt.cu"]
+    return ["post_weight_quantization_21_b200/csrc/hessian.cu", "post_weight_quantization_21_b200/csrc/hessian_tc.cu"]
 
 
 if __name__ == "__main__":

@@ -14,6 +14,13 @@ size_t hessian_simt_workspace(int64_t n_tokens, int64_t d);
 gptq_status hessian_simt_launch(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d, float* H,
                                 float scale, int32_t accumulate, void* workspace, cudaStream_t stream);
 
+// A1, tcgen05 tensor-core path for 16-bit inputs
+bool hessian_tc_supported(int64_t n_tokens, int64_t d, int32_t x_dtype);
+size_t hessian_tc_workspace(int64_t n_tokens, int64_t d);
+int hessian_tc_launches(int64_t n_tokens, int64_t d);
+gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d, float* H, float scale,
+                              int32_t accumulate, int32_t* status, void* workspace, cudaStream_t stream);
+
 // A2 + A3
 size_t prepare_workspace(int64_t d);
 gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,

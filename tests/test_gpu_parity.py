@@ -31,7 +31,12 @@ def _x(n, d, dtype, seed, corr=True):
     (1000, 200, torch.float32),      # ragged tile tail, ragged token tail
     (5000, 200, torch.bfloat16),
     (3000, 136, torch.float16),
-    (2048 * 9 + 17, 520, torch.bfloat16),
+    (2048 * 9 + 17, 520, torch.bfloat16),  # tensor-core path from here on: ragged 128/256 tiles
+    (4096, 256, torch.bfloat16),
+    (20000, 392, torch.float16),
+    (6144, 1024, torch.bfloat16),
+    (64, 384, torch.bfloat16),           # a single 64-token stage
+    (100, 512, torch.float16),           # one stage plus a ragged token tail
 ])
 def test_hessian_matches_oracle(n, d, dtype):
     X = _x(n, d, dtype, seed=n + d)
@@ -49,6 +54,14 @@ def test_hessian_accumulates_and_handles_empty_input():
     H0 = S.hessian(X[:0])                          # 0 tokens, overwrite mode: H = 0
     assert torch.count_nonzero(torch.triu(H0)) == 0
     S.hessian(X[:0], accumulate_into=H)            # 0 tokens, accumulate mode: unchanged
+    assert S.upper_rel_fro(H.cpu().numpy(), Href) <= S.H_REL_FRO
+
+
+def test_hessian_tensor_core_accumulate_mode():
+    X = _x(9000, 512, torch.bfloat16, seed=9).to(S.dev())
+    H = S.hessian(X[:5000])
+    S.hessian(X[5000:], accumulate_into=H)
+    Href = oracle.hessian(X.cpu().double().numpy())
     assert S.upper_rel_fro(H.cpu().numpy(), Href) <= S.H_REL_FRO
 
 
