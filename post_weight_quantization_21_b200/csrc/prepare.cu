@@ -4,22 +4,26 @@
 //
 // Route.  With J the index-reversal permutation, factor P = J Hd J = L L^T (ordinary lower
 // Cholesky) and invert Y = L^-1.  Then Hd = R R^T with R = J L J upper, and U = R^-1 = J Y J is upper
-// with U^T U = Hd^-1, so by uniqueness of the Cholesky factor U = chol(Hd^-1).  This needs one
-// factorisation and one triangular inversion (2/3 d^3 flops) instead of the pages' factorise /
-// invert / multiply / factorise route (4/3 d^3 flops); the oracle computes the pages' route.
+// with U^T U = Hd^-1, so by uniqueness of the Cholesky factor U = chol(Hd^-1).  One factorisation and
+// one triangular inversion (2/3 d^3 flops) replace the pages' factorise / invert / multiply /
+// factorise route (4/3 d^3 flops); the oracle computes the pages' route.
 //
-// Everything runs in place in the caller's U buffer:
-//   1. diag_mean      lambda = damp * mean(diag H)                              (1 CTA)
-//   2. reverse_damp   lower(P) = J (H + lambda I) J                              (from H's upper part)
-//   3. chol_step x D  right-looking blocked Cholesky, one launch per 64-column panel.  Launch j
-//                     applies panel j-1's rank-64 update to every tile right of it, and factors
-//                     panel j: every CTA of the panel recomputes the 64x64 diagonal block, so the
-//                     CTAs of a launch never wait on one another.  The diagonal blocks' inverses
-//                     go to the workspace.
-//   4. leaf_copy      diagonal blocks of P <- their inverses
-//   5. trtri levels   Y = L^-1 by doubling: [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]].
-//                     T = C A^-1 is parked transposed in P's unused upper triangle.
-//   6. rotate         U = J Y J (lower of the buffer -> upper), strict lower part zeroed.
+// One cooperative launch, one CTA (128 threads) per work item at a time, grid-wide barriers between
+// phases (bounded waits).  32x32 blocks, D = ceil(d / 32) block rows.  Everything lives in the
+// caller's U buffer ("P"): L (then Y) in the lower block triangle, the running right-hand sides R of
+// the inversion transposed in the upper block triangle.
+//   phase A   lambda = damp * mean(diag H)
+//   phase B   lower(P) = J (H + lambda I) J, upper(P) = 0
+//   phase j = 0..D  (each item independent of the others in its phase)
+//     panel     r = j..D-1: update P(r, j) and the diagonal block P(j, j) with panel j-1, factor the
+//               diagonal block and invert it (one warp, registers), L(r, j) = P(r, j) L(j,j)^-T.
+//               Every panel item refactors the 32x32 diagonal block, so no barrier separates the
+//               factorisation from the triangular solve.
+//     trailing  P(r, c) -= L(r, j-1) L(c, j-1)^T for j+1 <= c <= r
+//     inverse   Y(j-1, c) = L(j-1,j-1)^-1 R(j-1, c) (final row block of Y, written over L(j-1, c));
+//               R(i, c) -= L(i, j-1) Y(j-1, c) for i >= j.  (Right-looking block forward
+//               substitution of L Y = I, one block row behind the factorisation.)
+//   phase R   U = J Y J: lower block triangle -> upper, strict lower part zeroed.
 #include <math.h>
 
 #include "common.cuh"
@@ -28,374 +32,393 @@
 namespace gptq {
 namespace {
 
-constexpr int NB = 64;
-constexpr int LDS = NB + 1;
-constexpr int kThreads = 256;
+constexpr int NB = 32;
+constexpr int TS = 36;  // shared tile row stride (floats): rows stay 16-byte aligned
+constexpr int kThreads = 128;
+constexpr int kYChunk = 4;  // R updates per inverse item
+constexpr long long kWaitCycles = 4000000000LL;
 
-struct PrepPlan {
-  int D;  // 64-blocks per dimension
+struct PrepArgs {
+  const float* H;
+  float* P;
+  float* side;     // D inverse diagonal blocks, 32x32 row-major
+  float* lam;
+  unsigned* bar;   // [0] arrivals, [1] generation
+  int* abort_flag;
+  int32_t* status;
+  float damp;
+  int d, D;
 };
 
-PrepPlan prep_plan(int64_t d) { return PrepPlan{(int)((d + NB - 1) / NB)}; }
-
-// workspace layout: [0,256) lambda (float); [256, ...) D inverse diagonal blocks of 64x64 fp32
-size_t side_offset() { return 256; }
-
-__global__ void diag_mean_kernel(const float* __restrict__ H, int d, float damp, float* __restrict__ lam) {
-  double s = 0.0;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) s += (double)H[(size_t)i * d + i];
-  __shared__ double red[32];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+// ------------------------------------------------------------------ grid barrier (bounded)
+__device__ bool grid_barrier(const PrepArgs& a, unsigned& gen) {
+  __shared__ int s_ok;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    s = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned target = gen + 1;
+    __threadfence();
+    const unsigned arrived = atomicAdd(&a.bar[0], 1u);
+    if (arrived == gridDim.x - 1) {
+      atomicExch(&a.bar[0], 0u);
+      __threadfence();
+      atomicExch(&a.bar[1], target);
+    } else {
+      const long long t0 = clock64();
+      while (atomicAdd(&a.bar[1], 0u) != target) {
+        if (*(volatile int*)a.abort_flag) {
+          ok = 0;
+          break;
+        }
+        if (clock64() - t0 > kWaitCycles) {
+          *(volatile int*)a.abort_flag = 1;
+          report_status(a.status, GPTQ_ERR_TIMEOUT, -1);
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    gen = target;
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// ------------------------------------------------------------------ 32x32 tile helpers
+// Loads read through L2 (__ldcg): P is written by other CTAs during the launch.
+__device__ __forceinline__ float ldp(const float* p) { return __ldcg(p); }
+
+// S[r][c] = P(block) [r][c]; identity_pad puts 1 on the diagonal outside the matrix.
+__device__ void load_nat(float (*S)[TS], const float* P, int d, int br, int bc, bool identity_pad) {
+  for (int e = threadIdx.x; e < NB * NB; e += kThreads) {
+    const int r = e >> 5, c = e & 31;
+    const int gr = br * NB + r, gc = bc * NB + c;
+    S[r][c] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : ((identity_pad && r == c) ? 1.0f : 0.0f);
+  }
+}
+
+// S[c][r] = P(block) [r][c]
+__device__ void load_tr(float (*S)[TS], const float* P, int d, int br, int bc) {
+  for (int e = threadIdx.x; e < NB * NB; e += kThreads) {
+    const int r = e >> 5, c = e & 31;
+    const int gr = br * NB + r, gc = bc * NB + c;
+    S[c][r] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : 0.0f;
+  }
+}
+
+// S[c][r] = M[r][c] for a 32x32 row-major block M in global memory (the inverse diagonal blocks)
+__device__ void load_tr_block(float (*S)[TS], const float* M) {
+  for (int e = threadIdx.x; e < NB * NB; e += kThreads) S[e & 31][e >> 5] = ldp(M + e);
+}
+
+// Thread (ty, tx) owns rows 2ty, 2ty+1 and columns 4tx..4tx+3 of a 32x32 output.
+// acc[p][q] += sum_m Ak[m][2ty+p] * Bk[m][4tx+q]   (operands stored k-major)
+__device__ __forceinline__ void mma32(float acc[2][4], const float (*Ak)[TS], const float (*Bk)[TS], int ty,
+                                      int tx) {
+#pragma unroll 8
+  for (int m = 0; m < NB; ++m) {
+    const float2 av = *reinterpret_cast<const float2*>(&Ak[m][2 * ty]);
+    const float4 bv = *reinterpret_cast<const float4*>(&Bk[m][4 * tx]);
+    acc[0][0] = fmaf(av.x, bv.x, acc[0][0]);
+    acc[0][1] = fmaf(av.x, bv.y, acc[0][1]);
+    acc[0][2] = fmaf(av.x, bv.z, acc[0][2]);
+    acc[0][3] = fmaf(av.x, bv.w, acc[0][3]);
+    acc[1][0] = fmaf(av.y, bv.x, acc[1][0]);
+    acc[1][1] = fmaf(av.y, bv.y, acc[1][1]);
+    acc[1][2] = fmaf(av.y, bv.z, acc[1][2]);
+    acc[1][3] = fmaf(av.y, bv.w, acc[1][3]);
+  }
+}
+
+__device__ __forceinline__ void zero(float acc[2][4]) {
+#pragma unroll
+  for (int p = 0; p < 2; ++p)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[p][q] = 0.0f;
+}
+
+// Warp 0: factor the 32x32 block A (lower part, natural layout) and write its inverse transposed:
+// LiT[m][y] = L^-1[y][m].  Lane i keeps row i of A; lane c keeps column c of the right-hand sides
+// of L Y = I.  Right-looking with an unscaled pivot column:
+//   A[x][i] -= A[x][k] A[i][k] / A[k][k],   R[x][c] -= A[x][k] R[k][c] / A[k][k]   (x > k)
+// then L^-1[i][c] = R[i][c] / sqrt(pivot_i).  pivot_base: reversed-order index of the block's first
+// column, for the failure report.
+__device__ void warp_factor_invert(const float (*A)[TS], float (*LiT)[TS], float* colv, int d, int pivot_base,
+                                   int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  float a[NB], rr[NB], piv[NB];
+#pragma unroll
+  for (int c = 0; c < NB; ++c) {
+    a[c] = A[lane][c];
+    rr[c] = (c == lane) ? 1.0f : 0.0f;
+  }
+#pragma unroll
+  for (int k = 0; k < NB; ++k) {
+    float* cv = colv + (k & 1) * NB;
+    cv[lane] = a[k];
+    __syncwarp();
+    const float p = cv[k];
+    piv[k] = p;
+    if (lane == 0 && !(p > 0.0f && isfinite(p)) && pivot_base + k < d)
+      report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
+    const float inv = __frcp_rn(p);
+    const float li = a[k] * inv;
+    const float t = rr[k] * inv;
+#pragma unroll
+    for (int x = k + 1; x < NB; ++x) {
+      const float v = cv[x];
+      a[x] = fmaf(-li, v, a[x]);
+      rr[x] = fmaf(-v, t, rr[x]);
+    }
+  }
+  // column `lane` of L^-1 is row `lane` of LiT
+#pragma unroll
+  for (int i = 0; i < NB; ++i) LiT[lane][i] = (i >= lane) ? rr[i] / sqrtf(piv[i]) : 0.0f;
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
+  __shared__ __align__(16) float S0[NB][TS];
+  __shared__ __align__(16) float S1[NB][TS];
+  __shared__ __align__(16) float S2[NB][TS];
+  __shared__ __align__(16) float S3[NB][TS];
+  __shared__ __align__(16) float S4[NB][TS];
+  __shared__ float colv[2 * NB];
+  const int tid = threadIdx.x;
+  const int ty = tid >> 3, tx = tid & 7;
+  const int d = a.d, D = a.D;
+  float* P = a.P;
+  unsigned gen = 0;
+
+  // ---------------------------------------------------------------- phase A: lambda
+  if (blockIdx.x == 0) {
+    double s = 0.0;
+    for (int i = tid; i < d; i += kThreads) s += (double)a.H[(size_t)i * d + i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (threadIdx.x == 0) *lam = (float)((double)damp * s / (double)d);
-  }
-}
-
-// lower(P)[i][j] = H[d-1-i][d-1-j] (+lambda on the diagonal); 32x32 tiles, block (32, 8).
-__global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const float* __restrict__ lam,
-                                    float* __restrict__ P) {
-  if (blockIdx.x > blockIdx.y) return;
-  const float l = *lam;
-  const int j = blockIdx.x * 32 + threadIdx.x;
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int i = blockIdx.y * 32 + r;
-    if (i >= d || j >= d || j > i) continue;
-    float v = H[(size_t)(d - 1 - i) * d + (d - 1 - j)];
-    if (i == j) v += l;
-    P[(size_t)i * d + j] = v;
-  }
-}
-
-__device__ __forceinline__ void load_tile(float (*s)[LDS], const float* __restrict__ P, int d, int r0,
-                                          int c0, bool identity_pad) {
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    const int gr = r0 + r, gc = c0 + c;
-    float v;
-    if (gr < d && gc < d)
-      v = P[(size_t)gr * d + gc];
-    else
-      v = (identity_pad && r == c) ? 1.0f : 0.0f;
-    s[r][c] = v;
-  }
-}
-
-// acc[p][q] += sum_m A[ty*4+p][m] * B[tx*4+q][m]      (A B^T)
-__device__ __forceinline__ void tile_nt(float acc[4][4], const float (*A)[LDS], const float (*B)[LDS],
-                                        int ty, int tx, int m_lo = 0, int m_hi = NB) {
-  for (int m = m_lo; m < m_hi; ++m) {
-    float a[4], b[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) a[p] = A[ty * 4 + p][m];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) b[q] = B[tx * 4 + q][m];
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
-  }
-}
-
-// acc[p][q] += sum_m A[ty*4+p][m] * B[m][tx*4+q]      (A B)
-__device__ __forceinline__ void tile_nn(float acc[4][4], const float (*A)[LDS], const float (*B)[LDS],
-                                        int ty, int tx) {
-  for (int m = 0; m < NB; ++m) {
-    float a[4], b[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) a[p] = A[ty * 4 + p][m];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) b[q] = B[m][tx * 4 + q];
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
-  }
-}
-
-__device__ __forceinline__ void zero_acc(float acc[4][4]) {
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[p][q] = 0.f;
-}
-
-// In-smem Cholesky of the 64x64 block A (lower part) followed by its inverse Li (lower).
-// pivot_base: reversed-order index of A's first column (for the failure report).
-__device__ void factor_and_invert(float (*A)[LDS], float (*Li)[LDS], int d, int pivot_base,
-                                  int32_t* status) {
-  const int tid = threadIdx.x;
-  // right-looking with an unscaled pivot column: A[i][c] -= A[i][k] A[c][k] / A[k][k]
-  for (int k = 0; k < NB; ++k) {
-    const float piv = A[k][k];
-    if (tid == 0 && !(piv > 0.0f && isfinite(piv)))
-      report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
-    const float inv = 1.0f / piv;
-    for (int e = tid; e < NB * NB; e += kThreads) {
-      const int i = e / NB, c = e % NB;
-      if (c > k && c <= i) A[i][c] = fmaf(-A[i][k] * inv, A[c][k], A[i][c]);
-    }
+    __shared__ double red[kThreads / 32];
+    if ((tid & 31) == 0) red[tid >> 5] = s;
     __syncthreads();
-  }
-  // scale: L[i][c] = A[i][c] / sqrt(A[c][c]) for i >= c; zero above the diagonal
-  for (int e = tid; e < NB * NB; e += kThreads) {
-    const int i = e / NB, c = e % NB;
-    Li[i][c] = (c <= i) ? A[i][c] / sqrtf(A[c][c]) : 0.0f;
-  }
-  __syncthreads();
-  for (int e = tid; e < NB * NB; e += kThreads) {
-    const int i = e / NB, c = e % NB;
-    A[i][c] = Li[i][c];
-    Li[i][c] = (i == c) ? 1.0f : 0.0f;  // right-hand sides R = I
-  }
-  __syncthreads();
-  // forward substitution on all 64 right-hand sides: R[i][c] -= L[i][k] R[k][c] / L[k][k]
-  for (int k = 0; k < NB; ++k) {
-    const float inv = 1.0f / A[k][k];
-    for (int e = tid; e < NB * NB; e += kThreads) {
-      const int i = e / NB, c = e % NB;
-      if (i > k && c <= k) Li[i][c] = fmaf(-A[i][k] * inv, Li[k][c], Li[i][c]);
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < kThreads / 32; ++w) t += red[w];
+      *a.lam = (float)((double)a.damp * t / (double)d);
     }
-    __syncthreads();
   }
-  for (int e = tid; e < NB * NB; e += kThreads) {
-    const int i = e / NB, c = e % NB;
-    Li[i][c] = (c <= i) ? Li[i][c] / A[i][i] : 0.0f;
-  }
-  __syncthreads();
-}
+  if (!grid_barrier(a, gen)) return;
 
-__device__ __forceinline__ void tri_index(int t, int& rr, int& cc) {
-  // t -> (rr, cc) with 0 <= cc <= rr, row-major over the lower triangle
-  int r = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
-  while ((r + 1) * (r + 2) / 2 <= t) ++r;
-  while (r * (r + 1) / 2 > t) --r;
-  rr = r;
-  cc = t - r * (r + 1) / 2;
-}
-
-// One launch per panel j (see the file comment).  Blocks [0, D-j) factor the panel's row blocks;
-// the rest update the trailing lower tiles (r, c), j+1 <= c <= r < D, with panel j-1.
-__global__ void __launch_bounds__(kThreads) chol_step_kernel(float* __restrict__ P, int d, int D, int j,
-                                                              float* __restrict__ side,
-                                                              int32_t* __restrict__ status) {
-  extern __shared__ float smem[];
-  float(*S0)[LDS] = reinterpret_cast<float(*)[LDS]>(smem);
-  float(*S1)[LDS] = S0 + NB;
-  float(*S2)[LDS] = S1 + NB;
-  float(*S3)[LDS] = S2 + NB;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const int n_panel = D - j;
-  float acc[4][4];
-  if ((int)blockIdx.x < n_panel) {
-    const int r = j + blockIdx.x;
-    // S0: diagonal block (j, j) ; S1: L(j, j-1) ; S2: tile (r, j) ; S3: L(r, j-1)
-    load_tile(S0, P, d, j * NB, j * NB, true);
-    if (r > j) load_tile(S2, P, d, r * NB, j * NB, false);
-    if (j > 0) {
-      load_tile(S1, P, d, j * NB, (j - 1) * NB, false);
-      if (r > j) load_tile(S3, P, d, r * NB, (j - 1) * NB, false);
-    }
-    __syncthreads();
-    if (j > 0) {
-      zero_acc(acc);
-      tile_nt(acc, S1, S1, ty, tx);
-      float acc2[4][4];
-      zero_acc(acc2);
-      if (r > j) tile_nt(acc2, S3, S1, ty, tx);
-      __syncthreads();
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          S0[ty * 4 + p][tx * 4 + q] -= acc[p][q];
-          if (r > j) S2[ty * 4 + p][tx * 4 + q] -= acc2[p][q];
+  // ---------------------------------------------------------------- phase B: reversed, damped copy
+  {
+    const float lam = __ldcg(a.lam);
+    for (int i = blockIdx.x; i < d; i += gridDim.x) {
+      const float* src = a.H + (size_t)(d - 1 - i) * d + (d - 1);
+      float* dst = P + (size_t)i * d;
+      for (int j = tid; j < d; j += kThreads) {
+        float v = 0.0f;
+        if (j <= i) {
+          v = src[-j];
+          if (i == j) v += lam;
         }
+        dst[j] = v;
+      }
+    }
+  }
+  if (!grid_barrier(a, gen)) return;
+
+  // ---------------------------------------------------------------- phases 0..D
+  for (int j = 0; j <= D; ++j) {
+    const int n_panel = (j < D) ? D - j : 0;
+    const int n_trail = (j >= 1 && j < D) ? (D - j - 1) * (D - j) / 2 : 0;
+    const int rows_left = (j < D) ? D - j : 0;
+    const int chunks = (rows_left + kYChunk - 1) / kYChunk;
+    const int per_c = chunks > 0 ? chunks : 1;
+    const int n_inv = (j >= 1) ? j * per_c : 0;
+    const int n_items = n_panel + n_trail + n_inv;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      float acc[2][4], acc2[2][4];
+      if (it < n_panel) {
+        // ------------------------------------------------ panel item
+        const int r = j + it;
+        load_nat(S0, P, d, j, j, true);  // diagonal block
+        if (r > j) load_nat(S1, P, d, r, j, false);
+        if (j > 0) {
+          load_tr(S2, P, d, j, j - 1);  // L(j, j-1)^T
+          if (r > j) load_tr(S3, P, d, r, j - 1);
+        }
+        __syncthreads();
+        if (j > 0) {
+          zero(acc);
+          mma32(acc, S2, S2, ty, tx);
+          zero(acc2);
+          if (r > j) mma32(acc2, S3, S2, ty, tx);
+          __syncthreads();
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              S0[2 * ty + p][4 * tx + q] -= acc[p][q];
+              if (r > j) S1[2 * ty + p][4 * tx + q] -= acc2[p][q];
+            }
+        }
+        __syncthreads();
+        if (tid < 32) warp_factor_invert(S0, S4, colv, d, j * NB, a.status);
+        // S3 <- tile(r, j) transposed, for the triangular solve
+        if (r > j) {
+          for (int e = tid; e < NB * NB; e += kThreads) S3[e & 31][e >> 5] = S1[e >> 5][e & 31];
+        }
+        __syncthreads();
+        if (r == j) {
+          float* out = a.side + (size_t)j * NB * NB;  // natural layout: out[y][m] = S4[m][y]
+          for (int e = tid; e < NB * NB; e += kThreads) out[e] = S4[e & 31][e >> 5];
+        } else {
+          zero(acc);
+          mma32(acc, S3, S4, ty, tx);  // L(r, j) = tile(r, j) * Linv^T
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int gr = r * NB + 2 * ty + p, gc = j * NB + 4 * tx + q;
+              if (gr < d && gc < d) P[(size_t)gr * d + gc] = acc[p][q];
+            }
+        }
+      } else if (it < n_panel + n_trail) {
+        // ------------------------------------------------ trailing item
+        const int t = it - n_panel;
+        int rr = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
+        while ((rr + 1) * (rr + 2) / 2 <= t) ++rr;
+        while (rr * (rr + 1) / 2 > t) --rr;
+        const int cc = t - rr * (rr + 1) / 2;
+        const int r = j + 1 + rr, c = j + 1 + cc;
+        load_tr(S0, P, d, r, j - 1);
+        load_tr(S1, P, d, c, j - 1);
+        __syncthreads();
+        zero(acc);
+        mma32(acc, S0, S1, ty, tx);
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int gr = r * NB + 2 * ty + p, gc = c * NB + 4 * tx + q;
+            if (gr < d && gc < d) {
+              float* dst = P + (size_t)gr * d + gc;
+              *dst = ldp(dst) - acc[p][q];
+            }
+          }
+      } else {
+        // ------------------------------------------------ inverse item: column block c, rows chunk
+        const int t = it - n_panel - n_trail;
+        const int c = t / per_c, ch = t % per_c;
+        // Y(j-1, c) = Linv_{j-1} R(j-1, c);  R(j-1, j-1) = I, else R(j-1, c) sits transposed at P(c, j-1)
+        load_tr_block(S0, a.side + (size_t)(j - 1) * NB * NB);  // S0[m][x] = Linv[x][m]
+        if (c < j - 1) load_tr(S1, P, d, c, j - 1);            // S1[m][y] = R(j-1, c)[m][y]
+        __syncthreads();
+        if (c < j - 1) {
+          zero(acc);
+          mma32(acc, S0, S1, ty, tx);
+        } else {
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[p][q] = S0[4 * tx + q][2 * ty + p];
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) S2[2 * ty + p][4 * tx + q] = acc[p][q];  // Y natural
+        if (ch == 0) {
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int gr = (j - 1) * NB + 2 * ty + p, gc = c * NB + 4 * tx + q;
+              if (gr < d && gc < d) P[(size_t)gr * d + gc] = acc[p][q];
+            }
+        }
+        const int i0 = j + ch * kYChunk;
+        const int i1 = min(i0 + kYChunk, D);
+        for (int i = i0; i < i1; ++i) {
+          __syncthreads();
+          load_tr(S3, P, d, i, j - 1);  // S3[m][x] = L(i, j-1)[x][m]
+          __syncthreads();
+          zero(acc);
+          mma32(acc, S3, S2, ty, tx);
+          // R(i, c) is stored transposed at P(c, i)
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int x = 2 * ty + p, y = 4 * tx + q;
+              const int gr = c * NB + y, gc = i * NB + x;
+              if (gr < d && gc < d) {
+                float* dst = P + (size_t)gr * d + gc;
+                *dst = ldp(dst) - acc[p][q];
+              }
+            }
+        }
+      }
       __syncthreads();
     }
-    // S1 <- inverse of the factored diagonal block (S0 becomes L_jj)
-    factor_and_invert(S0, S1, d, j * NB, status);
-    if (r == j) {
-      float* out = side + (size_t)j * NB * NB;
-      for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) out[e] = S1[e / NB][e % NB];
-    } else {
-      // L(r, j) = tile(r, j) * Li^T
-      zero_acc(acc);
-      tile_nt(acc, S2, S1, ty, tx);
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int gr = r * NB + ty * 4 + p, gc = j * NB + tx * 4 + q;
-          if (gr < d && gc < d) P[(size_t)gr * d + gc] = acc[p][q];
-        }
-    }
-    return;
+    if (!grid_barrier(a, gen)) return;
   }
-  // trailing update with panel j-1
-  int rr, cc;
-  tri_index(blockIdx.x - n_panel, rr, cc);
-  const int r = j + 1 + rr, c = j + 1 + cc;
-  load_tile(S0, P, d, r * NB, (j - 1) * NB, false);
-  load_tile(S1, P, d, c * NB, (j - 1) * NB, false);
-  __syncthreads();
-  zero_acc(acc);
-  tile_nt(acc, S0, S1, ty, tx);
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int gr = r * NB + ty * 4 + p, gc = c * NB + tx * 4 + q;
-      if (gr < d && gc < d && gc <= gr) P[(size_t)gr * d + gc] -= acc[p][q];
-    }
-}
 
-__global__ void leaf_copy_kernel(float* __restrict__ P, int d, const float* __restrict__ side) {
-  const int j = blockIdx.x;
-  const float* src = side + (size_t)j * NB * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    const int gr = j * NB + r, gc = j * NB + c;
-    if (gr < d && gc < d) P[(size_t)gr * d + gc] = (c <= r) ? src[e] : 0.0f;
+  // ---------------------------------------------------------------- phase R: U = J Y J in place
+  for (int i = blockIdx.x; i < d; i += gridDim.x) {
+    float* row = P + (size_t)i * d;
+    float* mirror = P + (size_t)(d - 1 - i) * d + (d - 1);
+    for (int j = tid; j <= i; j += kThreads) {
+      if (j < i) {
+        mirror[-j] = ldp(row + j);
+        row[j] = 0.0f;
+      } else if (i < d - 1 - i) {  // diagonal pair (i, i) <-> (d-1-i, d-1-i)
+        const float va = ldp(row + i), vb = ldp(mirror - i);
+        row[i] = vb;
+        mirror[-i] = va;
+      }
+    }
   }
 }
 
-// Level with g-block halves.  Pair p: A = blocks [a0, a0+g), B = [a0+g, min(a0+2g, D)).
-// T tile (r, c) (r in B, c in A) = sum_{k=c}^{a0+g-1} C(r, k) * Ainv(k, c), stored transposed at
-// block (c, r) of the upper triangle.
-__global__ void __launch_bounds__(kThreads) trtri_t_kernel(float* __restrict__ P, int d, int D, int g) {
-  extern __shared__ float smem[];
-  float(*Cs)[LDS] = reinterpret_cast<float(*)[LDS]>(smem);
-  float(*As)[LDS] = Cs + NB;
-  const int per_pair = g * g;  // upper bound of tiles per pair (B may be shorter)
-  const int p = blockIdx.x / per_pair, t = blockIdx.x % per_pair;
-  const int a0 = p * 2 * g, b0 = a0 + g;
-  const int b1 = min(a0 + 2 * g, D);
-  const int r = b0 + t / g, c = a0 + t % g;
-  if (r >= b1) return;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4];
-  zero_acc(acc);
-  for (int k = c; k < a0 + g; ++k) {
-    load_tile(Cs, P, d, r * NB, k * NB, false);
-    load_tile(As, P, d, k * NB, c * NB, false);
-    __syncthreads();
-    tile_nn(acc, Cs, As, ty, tx);
-    __syncthreads();
-  }
-#pragma unroll
-  for (int pp = 0; pp < 4; ++pp)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int x = ty * 4 + pp, y = tx * 4 + q;  // T[x][y] -> P[c*NB + y][r*NB + x]
-      const int gr = c * NB + y, gc = r * NB + x;
-      if (gr < d && gc < d) P[(size_t)gr * d + gc] = acc[pp][q];
-    }
-}
-
-// Y tile (r, c) = - sum_{k=b0}^{r} Binv(r, k) * T(k, c), written over C(r, c).
-__global__ void __launch_bounds__(kThreads) trtri_y_kernel(float* __restrict__ P, int d, int D, int g) {
-  extern __shared__ float smem[];
-  float(*Bs)[LDS] = reinterpret_cast<float(*)[LDS]>(smem);
-  float(*Ts)[LDS] = Bs + NB;
-  const int per_pair = g * g;
-  const int p = blockIdx.x / per_pair, t = blockIdx.x % per_pair;
-  const int a0 = p * 2 * g, b0 = a0 + g;
-  const int b1 = min(a0 + 2 * g, D);
-  const int r = b0 + t / g, c = a0 + t % g;
-  if (r >= b1) return;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4];
-  zero_acc(acc);
-  for (int k = b0; k <= r; ++k) {
-    load_tile(Bs, P, d, r * NB, k * NB, false);
-    load_tile(Ts, P, d, c * NB, k * NB, false);  // holds T(k, c) transposed
-    __syncthreads();
-    tile_nt(acc, Bs, Ts, ty, tx);
-    __syncthreads();
-  }
-#pragma unroll
-  for (int pp = 0; pp < 4; ++pp)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int gr = r * NB + ty * 4 + pp, gc = c * NB + tx * 4 + q;
-      if (gr < d && gc < d) P[(size_t)gr * d + gc] = -acc[pp][q];
-    }
-}
-
-// U = J Y J: buffer[d-1-i][d-1-j] <- buffer[i][j] for i > j, buffer[i][j] <- 0; diagonal reversed.
-__global__ void rotate_kernel(float* __restrict__ P, int d) {
-  if (blockIdx.x > blockIdx.y) return;
-  const int j = blockIdx.x * 32 + threadIdx.x;
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int i = blockIdx.y * 32 + r;
-    if (i >= d || j >= d || j > i) continue;
-    if (i > j) {
-      const float v = P[(size_t)i * d + j];
-      P[(size_t)(d - 1 - i) * d + (d - 1 - j)] = v;
-      P[(size_t)i * d + j] = 0.0f;
-    } else if (i < d - 1 - i) {
-      const size_t a = (size_t)i * d + i, b = (size_t)(d - 1 - i) * d + (d - 1 - i);
-      const float va = P[a], vb = P[b];
-      P[a] = vb;
-      P[b] = va;
-    }
-  }
-}
+constexpr size_t kSideOffset = 256;
 
 }  // namespace
 
 size_t prepare_workspace(int64_t d) {
-  PrepPlan p = prep_plan(d);
-  return side_offset() + (size_t)p.D * NB * NB * sizeof(float);
+  const int64_t D = (d + NB - 1) / NB;
+  return kSideOffset + (size_t)D * NB * NB * sizeof(float);
 }
 
-gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status,
-                           void* workspace, cudaStream_t stream) {
+gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status, void* workspace,
+                           cudaStream_t stream) {
   const int d = (int)d64;
-  PrepPlan pl = prep_plan(d);
-  const int D = pl.D;
   char* ws = static_cast<char*>(workspace);
-  float* lam = reinterpret_cast<float*>(ws);
-  float* side = reinterpret_cast<float*>(ws + side_offset());
-  static bool attr_done = false;
-  const int smem4 = 4 * NB * LDS * sizeof(float);
-  const int smem2 = 2 * NB * LDS * sizeof(float);
-  if (!attr_done) {
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem4));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(trtri_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(trtri_y_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2));
-    attr_done = true;
-  }
+  PrepArgs a;
+  a.H = H;
+  a.P = U;
+  a.lam = reinterpret_cast<float*>(ws);
+  a.bar = reinterpret_cast<unsigned*>(ws + 64);
+  a.abort_flag = reinterpret_cast<int*>(ws + 128);
+  a.side = reinterpret_cast<float*>(ws + kSideOffset);
+  a.status = status;
+  a.damp = damp;
+  a.d = d;
+  a.D = (d + NB - 1) / NB;
+  int dev = 0, sms = 0, occ = 0, coop = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+  if (!coop) return GPTQ_ERR_CUDA;
+  GPTQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prepare_kernel, kThreads, 0));
+  if (occ < 1) return GPTQ_ERR_CUDA;
+  const int grid = sms * (occ < 2 ? occ : 2);
   GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), stream));
-  diag_mean_kernel<<<1, 1024, 0, stream>>>(H, d, damp, lam);
-  GPTQ_LAUNCH_CHECK();
-  const int D32 = (d + 31) / 32;
-  reverse_damp_kernel<<<dim3(D32, D32), dim3(32, 8), 0, stream>>>(H, d, lam, U);
-  GPTQ_LAUNCH_CHECK();
-  for (int j = 0; j < D; ++j) {
-    int n = D - j;
-    if (j > 0) n += (D - j - 1) * (D - j) / 2;
-    chol_step_kernel<<<n, kThreads, smem4, stream>>>(U, d, D, j, side, status);
-    GPTQ_LAUNCH_CHECK();
-  }
-  leaf_copy_kernel<<<D, kThreads, 0, stream>>>(U, d, side);
-  GPTQ_LAUNCH_CHECK();
-  for (int g = 1; g < D; g *= 2) {
-    const int pairs = (D + 2 * g - 1) / (2 * g);
-    const int n = pairs * g * g;
-    trtri_t_kernel<<<n, kThreads, smem2, stream>>>(U, d, D, g);
-    GPTQ_LAUNCH_CHECK();
-    trtri_y_kernel<<<n, kThreads, smem2, stream>>>(U, d, D, g);
-    GPTQ_LAUNCH_CHECK();
-  }
-  rotate_kernel<<<dim3(D32, D32), dim3(32, 8), 0, stream>>>(U, d);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_CUDA_TRY(cudaMemsetAsync(ws + 64, 0, 128, stream));  // barrier words and abort flag
+  void* args[] = {&a};
+  GPTQ_CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(prepare_kernel), dim3(grid), dim3(kThreads),
+                                            args, 0, stream));
+  count_launch();
   return GPTQ_OK;
 }
 

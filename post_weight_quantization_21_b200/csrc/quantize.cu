@@ -47,51 +47,28 @@ __global__ void __launch_bounds__(256) convert_rowgrid_kernel(const T* __restric
   }
 }
 
-// Column loop over block [i1, i1 + 32*NS) for 8 rows per CTA.
+// Column loop of one row over block [i1, i1 + 32*NS), run by one warp.  v[s] holds column
+// i1 + 32*s + lane of the row (current values).  Us is the block's corner of U (strict upper part,
+// row-major B x B) and invd the reciprocals of its diagonal.  Each step broadcasts w_i from its
+// lane, rounds it, and applies err_i * U[i, j] to the columns of the block.  The inner loop is not
+// unrolled: one copy of the step per register slot keeps the code small enough for the i-cache.
 template <int NS>
-__global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
-                                                      const float* __restrict__ U, int bits,
-                                                      int group_size, uint8_t* __restrict__ codes,
-                                                      float* __restrict__ scales,
-                                                      int32_t* __restrict__ zeros,
-                                                      float* __restrict__ err_out) {
+__device__ __forceinline__ void column_loop(float (&v)[NS], const float* __restrict__ Us,
+                                            const float* __restrict__ invd, int i1, int group_size,
+                                            int n_groups, float maxq, float& scale, float& zero,
+                                            const float* wrow, int64_t row, float* __restrict__ scales,
+                                            int32_t* __restrict__ zeros, uint32_t (&code_reg)[NS],
+                                            float (&err_reg)[NS]) {
   constexpr int B = 32 * NS;
-  extern __shared__ float sm[];
-  float* Us = sm;           // [B][B], strict lower part zero
-  float* invd = sm + B * B;  // [B]
-  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
-    const int r = e / B, c = e % B;
-    Us[e] = (c > r) ? U[(size_t)(i1 + r) * d + i1 + c] : 0.0f;
-  }
-  for (int r = threadIdx.x; r < B; r += blockDim.x) invd[r] = 1.0f / U[(size_t)(i1 + r) * d + i1 + r];
-  __syncthreads();
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
-  if (row >= m) return;
-  float* wr = w + row * d;
-  float v[NS];
-#pragma unroll
-  for (int s = 0; s < NS; ++s) v[s] = wr[i1 + s * 32 + lane];
-  const float maxq = (float)((1 << bits) - 1);
-  const int n_groups = group_size ? d / group_size : 1;
-  float scale = 0.f, zero = 0.f;
-  if (group_size == 0) {
-    scale = scales[row];
-    zero = (float)zeros[row];
-  } else if (i1 % group_size != 0) {  // block inside a group that started in an earlier block
-    scale = scales[row * n_groups + i1 / group_size];
-    zero = (float)zeros[row * n_groups + i1 / group_size];
-  }
-  uint32_t code_reg[NS];
-  float err_reg[NS];
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
-#pragma unroll
+#pragma unroll 1
     for (int l = 0; l < 32; ++l) {
       const int i = s * 32 + l;
-      if (l == 0 && group_size != 0 && ((i1 + i) % group_size) == 0) {
+      if (group_size != 0 && l == 0 && ((i1 + i) % group_size) == 0) {
         // grid of the group starting here, from the current values of its columns
-        const int gw = group_size / 32;  // slots covered inside the block
+        const int gw = group_size / 32;  // register slots the group covers inside the block
         float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
         for (int t = 0; t < NS; ++t)
@@ -99,8 +76,8 @@ __global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int
             mn = fminf(mn, v[t]);
             mx = fmaxf(mx, v[t]);
           }
-        for (int c = i1 + B + lane; c < i1 + i + group_size; c += 32) {  // group wider than block
-          const float x = wr[c];
+        for (int c = i1 + B + lane; c < i1 + i + group_size; c += 32) {  // group wider than the block
+          const float x = wrow[c];
           mn = fminf(mn, x);
           mx = fmaxf(mx, x);
         }
@@ -127,10 +104,167 @@ __global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int
       for (int t = 0; t < NS; ++t) v[t] = fmaf(-err, urow[t * 32 + lane], v[t]);
     }
   }
+}
+
+// Grid state of a row at the start of block i1.
+__device__ __forceinline__ void grid_at_block(int64_t row, int i1, int group_size, int n_groups,
+                                              const float* scales, const int32_t* zeros, float& scale,
+                                              float& zero) {
+  if (group_size == 0) {
+    scale = scales[row];
+    zero = (float)zeros[row];
+  } else if (i1 % group_size != 0) {  // block inside a group that started in an earlier block
+    scale = scales[row * n_groups + i1 / group_size];
+    zero = (float)zeros[row * n_groups + i1 / group_size];
+  } else {
+    scale = 1.0f;
+    zero = 0.0f;
+  }
+}
+
+// Loads U[i1:i1+B, i1:i1+B] (strict upper part) and the reciprocals of its diagonal.
+template <int B>
+__device__ __forceinline__ void load_u_block(float* Us, float* invd, const float* __restrict__ U, int d, int i1) {
+  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
+    const int r = e / B, c = e % B;
+    Us[e] = (c > r) ? U[(size_t)(i1 + r) * d + i1 + c] : 0.0f;
+  }
+  for (int r = threadIdx.x; r < B; r += blockDim.x) invd[r] = 1.0f / U[(size_t)(i1 + r) * d + i1 + r];
+}
+
+// Column loop over block [i1, i1 + 32*NS) for 8 rows per CTA (per-block launch path).
+template <int NS>
+__global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
+                                                      const float* __restrict__ U, int bits,
+                                                      int group_size, uint8_t* __restrict__ codes,
+                                                      float* __restrict__ scales,
+                                                      int32_t* __restrict__ zeros,
+                                                      float* __restrict__ err_out) {
+  constexpr int B = 32 * NS;
+  extern __shared__ float sm[];
+  float* Us = sm;
+  float* invd = sm + B * B;
+  load_u_block<B>(Us, invd, U, d, i1);
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
+  if (row >= m) return;
+  float* wr = w + row * d;
+  float v[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) v[s] = wr[i1 + s * 32 + lane];
+  const float maxq = (float)((1 << bits) - 1);
+  const int n_groups = group_size ? d / group_size : 1;
+  float scale, zero;
+  grid_at_block(row, i1, group_size, n_groups, scales, zeros, scale, zero);
+  uint32_t code_reg[NS];
+  float err_reg[NS];
+  column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, wr, row, scales, zeros, code_reg,
+                  err_reg);
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
     codes[row * d + i1 + s * 32 + lane] = (uint8_t)code_reg[s];
     err_out[row * B + s * 32 + lane] = err_reg[s];
+  }
+}
+
+// Whole quantization of 8 rows per CTA in one launch (layers whose U stays in L2): for every block,
+// the column loop (one warp per row, U corner in shared memory), then the lazy update of the CTA's
+// rows, W[rows, i2:] -= Err[rows, :] U[i1:i2, i2:], with U streamed through shared memory in
+// 128-column chunks.  Rows are independent given U, so CTAs never wait on one another.
+template <typename T, int NS>
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ W, int64_t m, int d,
+                                                            const float* __restrict__ U, int bits,
+                                                            int group_size, float* __restrict__ w,
+                                                            uint8_t* __restrict__ codes,
+                                                            float* __restrict__ scales,
+                                                            int32_t* __restrict__ zeros) {
+  constexpr int B = 32 * NS;
+  constexpr int CW = 128;  // lazy-update chunk width (columns)
+  extern __shared__ __align__(16) float sm[];
+  float* Us = sm;                // [B][B] corner of U, then [B][CW] chunks of the U panel
+  float* invd = sm + B * CW;     // [B]
+  float* errs = invd + B;        // [8][B]
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
+  const bool valid = row < m;
+  const float maxq = (float)((1 << bits) - 1);
+  const int n_groups = group_size ? d / group_size : 1;
+  float* wr = w + (valid ? row : 0) * d;
+  if (valid) {
+    const T* src = W + row * d;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int c = lane; c < d; c += 32) {
+      const float x = to_f32(src[c]);
+      wr[c] = x;
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    if (group_size == 0) {
+      mn = warp_min(mn);
+      mx = warp_max(mx);
+      if (lane == 0) {
+        float s, z;
+        grid_from_range(mn, mx, maxq, s, z);
+        scales[row] = s;
+        zeros[row] = (int32_t)z;
+      }
+    }
+  }
+  float scale = 1.0f, zero = 0.0f;
+  for (int i1 = 0; i1 < d; i1 += B) {
+    __syncthreads();
+    load_u_block<B>(Us, invd, U, d, i1);
+    __syncthreads();
+    if (valid) {
+      __syncwarp();
+      if (i1 == 0 || group_size == 0) {
+        grid_at_block(row, i1, group_size, n_groups, scales, zeros, scale, zero);
+      }
+      float v[NS];
+#pragma unroll
+      for (int s = 0; s < NS; ++s) v[s] = wr[i1 + s * 32 + lane];
+      uint32_t code_reg[NS];
+      float err_reg[NS];
+      column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, wr, row, scales, zeros,
+                      code_reg, err_reg);
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        codes[row * d + i1 + s * 32 + lane] = (uint8_t)code_reg[s];
+        errs[warp * B + s * 32 + lane] = err_reg[s];
+      }
+    }
+    // lazy update of this CTA's rows over the columns after the block
+    for (int c0 = i1 + B; c0 < d; c0 += CW) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < B * CW / 4; e += blockDim.x) {
+        const int k = e / (CW / 4), c = (e % (CW / 4)) * 4;
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c0 + c < d) u = *reinterpret_cast<const float4*>(U + (size_t)(i1 + k) * d + c0 + c);
+        *reinterpret_cast<float4*>(Us + k * CW + c) = u;
+      }
+      __syncthreads();
+      if (valid && c0 + 4 * lane < d) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* er = errs + warp * B;
+#pragma unroll 8
+        for (int k = 0; k < B; ++k) {
+          const float e = er[k];
+          const float4 u = *reinterpret_cast<const float4*>(Us + k * CW + 4 * lane);
+          acc.x = fmaf(e, u.x, acc.x);
+          acc.y = fmaf(e, u.y, acc.y);
+          acc.z = fmaf(e, u.z, acc.z);
+          acc.w = fmaf(e, u.w, acc.w);
+        }
+        float4* dst = reinterpret_cast<float4*>(wr + c0 + 4 * lane);
+        float4 o = *dst;
+        o.x -= acc.x;
+        o.y -= acc.y;
+        o.z -= acc.z;
+        o.w -= acc.w;
+        *dst = o;
+      }
+    }
   }
 }
 
@@ -230,11 +364,38 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
   return GPTQ_OK;
 }
 
+template <typename T, int NS>
+gptq_status launch_rows(const void* W, int64_t m, int d, const float* U, int bits, int gs, float* ww, uint8_t* codes,
+                        float* scales, int32_t* zeros, cudaStream_t s) {
+  constexpr int B = 32 * NS;
+  const int smem = (B * 128 + B + kRowsPerCta * B) * sizeof(float);
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(quantize_rows_kernel<T, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int grid = (int)((m + kRowsPerCta - 1) / kRowsPerCta);
+  quantize_rows_kernel<T, NS><<<grid, 256, smem, s>>>(static_cast<const T*>(W), m, d, U, bits, gs, ww, codes, scales,
+                                                      zeros);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+template <typename T>
+gptq_status launch_rows_b(const void* W, int64_t m, int d, const float* U, const gptq_quant_cfg& cfg, float* ww,
+                          uint8_t* codes, float* scales, int32_t* zeros, cudaStream_t s) {
+  switch (cfg.block_size) {
+    case 32: return launch_rows<T, 1>(W, m, d, U, cfg.bits, cfg.group_size, ww, codes, scales, zeros, s);
+    case 64: return launch_rows<T, 2>(W, m, d, U, cfg.bits, cfg.group_size, ww, codes, scales, zeros, s);
+    case 128: return launch_rows<T, 4>(W, m, d, U, cfg.bits, cfg.group_size, ww, codes, scales, zeros, s);
+    default: return GPTQ_ERR_ARG;
+  }
+}
+
 }  // namespace
 
 size_t quantize_workspace(int64_t m, int64_t d, int block_size) {
   return align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * block_size * sizeof(float), 256);
 }
+
+// U of up to 4096^2 fp32 (64 MB) stays in the 126 MB L2, so each CTA can stream it for its own rows.
+bool quantize_fused(int64_t d) { return d <= 4096; }
 
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d64, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
@@ -243,6 +404,14 @@ gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d
   char* ws = static_cast<char*>(workspace);
   float* ww = reinterpret_cast<float*>(ws);
   float* err = reinterpret_cast<float*>(ws + align_up((size_t)m * d * sizeof(float), 256));
+  if (quantize_fused(d)) {
+    switch (w_dtype) {
+      case GPTQ_FP32: return launch_rows_b<float>(W, m, d, U, cfg, ww, codes, scales, zeros, s);
+      case GPTQ_FP16: return launch_rows_b<__half>(W, m, d, U, cfg, ww, codes, scales, zeros, s);
+      case GPTQ_BF16: return launch_rows_b<__nv_bfloat16>(W, m, d, U, cfg, ww, codes, scales, zeros, s);
+      default: return GPTQ_ERR_ARG;
+    }
+  }
   switch (w_dtype) {
     case GPTQ_FP32: launch_convert<float>(W, m, d, cfg.bits, cfg.group_size, ww, scales, zeros, s); break;
     case GPTQ_FP16: launch_convert<__half>(W, m, d, cfg.bits, cfg.group_size, ww, scales, zeros, s); break;

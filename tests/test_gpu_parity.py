@@ -74,7 +74,7 @@ def test_hessian_full_size_opt125m_layer():
 
 
 # ------------------------------------------------------------------------------------------ A2 + A3
-@pytest.mark.parametrize("d", [1, 5, 64, 128, 200, 768, 1000])
+@pytest.mark.parametrize("d", [1, 5, 31, 33, 64, 128, 200, 768, 1000, 2048, 4224])
 def test_prepare_matches_oracle(d):
     n = max(4 * d, 64)
     X = _x(n, d, torch.float64, seed=d)
@@ -111,6 +111,8 @@ QUANT_CASES = [
     (64, 512, 4, 256, 128),
     (48, 384, 4, 64, 32),
     (1, 128, 4, 0, 128),
+    (40, 4224, 3, 128, 128),   # wider than 4096: per-block launches instead of the fused kernel
+    (24, 4352, 4, 0, 64),
 ]
 
 
