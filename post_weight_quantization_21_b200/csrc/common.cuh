@@ -48,9 +48,11 @@ template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // Asymmetric min/max grid: the range widened to contain 0, an empty range becomes [-1, 1];
-// scale = (hi - lo) / maxq and zero = rint(-lo / scale), both in IEEE fp32.
+// scale = (hi - lo) / maxq in IEEE fp32, rscale = IEEE fp32 reciprocal of scale, and
+// zero = rint(-lo * rscale).  Quotients that decide an integer are always formed as x * rscale
+// (IEEE fp32 product, not contracted into an FMA).
 __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, float& scale,
-                                                float& zero) {
+                                                float& zero, float& rscale) {
   float lo = fminf(mn, 0.0f);
   float hi = fmaxf(mx, 0.0f);
   if (lo == hi) {
@@ -58,7 +60,8 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, 
     hi = 1.0f;
   }
   scale = __fdiv_rn(hi - lo, maxq);
-  zero = rintf(__fdiv_rn(-lo, scale));
+  rscale = __frcp_rn(scale);
+  zero = rintf(__fmul_rn(-lo, rscale));
 }
 
 __device__ __forceinline__ float warp_min(float v) {

@@ -43,7 +43,7 @@ struct PrepArgs {
   float* P;
   float* side;     // D inverse diagonal blocks, 32x32 row-major
   float* lam;
-  unsigned* bar;   // [0] arrivals, [1] generation
+  unsigned* bar;   // [0] arrivals, [32] generation (separate 128-byte lines)
   int* abort_flag;
   int32_t* status;
   float damp;
@@ -51,21 +51,32 @@ struct PrepArgs {
 };
 
 // ------------------------------------------------------------------ grid barrier (bounded)
+// Arrival counter and generation word sit in different 128-byte lines; waiters poll the generation
+// with acquire loads (no read-modify-write traffic on the line the arrivals update).
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ bool grid_barrier(const PrepArgs& a, unsigned& gen) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
     const unsigned target = gen + 1;
+    unsigned* count = a.bar;
+    unsigned* generation = a.bar + 32;
     __threadfence();
-    const unsigned arrived = atomicAdd(&a.bar[0], 1u);
+    const unsigned arrived = atomicAdd(count, 1u);
     if (arrived == gridDim.x - 1) {
-      atomicExch(&a.bar[0], 0u);
+      *(volatile unsigned*)count = 0u;
       __threadfence();
-      atomicExch(&a.bar[1], target);
+      atomicExch(generation, target);
     } else {
       const long long t0 = clock64();
-      while (atomicAdd(&a.bar[1], 0u) != target) {
+      unsigned ns = 32;
+      while (ld_acquire(generation) != target) {
         if (*(volatile int*)a.abort_flag) {
           ok = 0;
           break;
@@ -76,7 +87,8 @@ __device__ bool grid_barrier(const PrepArgs& a, unsigned& gen) {
           ok = 0;
           break;
         }
-        __nanosleep(64);
+        __nanosleep(ns);
+        if (ns < 256) ns *= 2;
       }
     }
     __threadfence();
@@ -91,27 +103,47 @@ __device__ bool grid_barrier(const PrepArgs& a, unsigned& gen) {
 // Loads read through L2 (__ldcg): P is written by other CTAs during the launch.
 __device__ __forceinline__ float ldp(const float* p) { return __ldcg(p); }
 
-// S[r][c] = P(block) [r][c]; identity_pad puts 1 on the diagonal outside the matrix.
-__device__ void load_nat(float (*S)[TS], const float* P, int d, int br, int bc, bool identity_pad) {
-  for (int e = threadIdx.x; e < NB * NB; e += kThreads) {
+// A 32x32 block held in registers, 8 values per thread: element e = tid + 128 k sits at row e / 32,
+// column e % 32 (each warp reads whole rows, coalesced).  fetch() issues all 8 loads before any is
+// used, so a tile costs one L2 round trip; put_*() store it to shared memory.
+struct TileRegs {
+  float v[8];
+};
+
+__device__ __forceinline__ TileRegs fetch(const float* P, int d, int br, int bc, bool identity_pad = false) {
+  TileRegs t;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = threadIdx.x + kThreads * k;
     const int r = e >> 5, c = e & 31;
     const int gr = br * NB + r, gc = bc * NB + c;
-    S[r][c] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : ((identity_pad && r == c) ? 1.0f : 0.0f);
+    t.v[k] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : ((identity_pad && r == c) ? 1.0f : 0.0f);
+  }
+  return t;
+}
+
+// A 32x32 row-major block M in global memory (the inverse diagonal blocks)
+__device__ __forceinline__ TileRegs fetch_block(const float* M) {
+  TileRegs t;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) t.v[k] = ldp(M + threadIdx.x + kThreads * k);
+  return t;
+}
+
+__device__ __forceinline__ void put_nat(float (*S)[TS], const TileRegs& t) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = threadIdx.x + kThreads * k;
+    S[e >> 5][e & 31] = t.v[k];
   }
 }
 
-// S[c][r] = P(block) [r][c]
-__device__ void load_tr(float (*S)[TS], const float* P, int d, int br, int bc) {
-  for (int e = threadIdx.x; e < NB * NB; e += kThreads) {
-    const int r = e >> 5, c = e & 31;
-    const int gr = br * NB + r, gc = bc * NB + c;
-    S[c][r] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : 0.0f;
+__device__ __forceinline__ void put_tr(float (*S)[TS], const TileRegs& t) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = threadIdx.x + kThreads * k;
+    S[e & 31][e >> 5] = t.v[k];
   }
-}
-
-// S[c][r] = M[r][c] for a 32x32 row-major block M in global memory (the inverse diagonal blocks)
-__device__ void load_tr_block(float (*S)[TS], const float* M) {
-  for (int e = threadIdx.x; e < NB * NB; e += kThreads) S[e & 31][e >> 5] = ldp(M + e);
 }
 
 // Thread (ty, tx) owns rows 2ty, 2ty+1 and columns 4tx..4tx+3 of a 32x32 output.
@@ -143,13 +175,14 @@ __device__ __forceinline__ void zero(float acc[2][4]) {
 // Warp 0: factor the 32x32 block A (lower part, natural layout) and write its inverse transposed:
 // LiT[m][y] = L^-1[y][m].  Lane i keeps row i of A; lane c keeps column c of the right-hand sides
 // of L Y = I.  Right-looking with an unscaled pivot column:
-//   A[x][i] -= A[x][k] A[i][k] / A[k][k],   R[x][c] -= A[x][k] R[k][c] / A[k][k]   (x > k)
-// then L^-1[i][c] = R[i][c] / sqrt(pivot_i).  pivot_base: reversed-order index of the block's first
-// column, for the failure report.
-__device__ void warp_factor_invert(const float (*A)[TS], float (*LiT)[TS], float* colv, int d, int pivot_base,
-                                   int32_t* status) {
+//   A[i][x] -= A[i][k] A[x][k] / A[k][k],   R[x][c] -= A[x][k] R[k][c] / A[k][k]   (x > k)
+// then L^-1[i][c] = R[i][c] / sqrt(pivot_i).  The pivot column is shared through shared memory
+// (zeros at and above the pivot) and read four entries at a time.  pivot_base: reversed-order index
+// of the block's first column, for the failure report.
+__device__ void warp_factor_invert(const float (*A)[TS], float (*LiT)[TS], float* colv, float* rsm, int d,
+                                   int pivot_base, int32_t* status) {
   const int lane = threadIdx.x & 31;
-  float a[NB], rr[NB], piv[NB];
+  float a[NB], rr[NB];
 #pragma unroll
   for (int c = 0; c < NB; ++c) {
     a[c] = A[lane][c];
@@ -158,25 +191,33 @@ __device__ void warp_factor_invert(const float (*A)[TS], float (*LiT)[TS], float
 #pragma unroll
   for (int k = 0; k < NB; ++k) {
     float* cv = colv + (k & 1) * NB;
-    cv[lane] = a[k];
+    cv[lane] = (lane > k) ? a[k] : 0.0f;
+    const float p = __shfl_sync(0xffffffffu, a[k], k);
     __syncwarp();
-    const float p = cv[k];
-    piv[k] = p;
-    if (lane == 0 && !(p > 0.0f && isfinite(p)) && pivot_base + k < d)
-      report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
-    const float inv = __frcp_rn(p);
+    const float inv = __fdividef(1.0f, p);
     const float li = a[k] * inv;
     const float t = rr[k] * inv;
+    if (lane == 0) {
+      rsm[k] = rsqrtf(p);
+      if (!(p > 0.0f && isfinite(p)) && pivot_base + k < d) report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
+    }
 #pragma unroll
-    for (int x = k + 1; x < NB; ++x) {
-      const float v = cv[x];
-      a[x] = fmaf(-li, v, a[x]);
-      rr[x] = fmaf(-v, t, rr[x]);
+    for (int x4 = (k + 1) & ~3; x4 < NB; x4 += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(cv + x4);
+      a[x4 + 0] = fmaf(-li, v.x, a[x4 + 0]);
+      a[x4 + 1] = fmaf(-li, v.y, a[x4 + 1]);
+      a[x4 + 2] = fmaf(-li, v.z, a[x4 + 2]);
+      a[x4 + 3] = fmaf(-li, v.w, a[x4 + 3]);
+      rr[x4 + 0] = fmaf(-v.x, t, rr[x4 + 0]);
+      rr[x4 + 1] = fmaf(-v.y, t, rr[x4 + 1]);
+      rr[x4 + 2] = fmaf(-v.z, t, rr[x4 + 2]);
+      rr[x4 + 3] = fmaf(-v.w, t, rr[x4 + 3]);
     }
   }
+  __syncwarp();
   // column `lane` of L^-1 is row `lane` of LiT
 #pragma unroll
-  for (int i = 0; i < NB; ++i) LiT[lane][i] = (i >= lane) ? rr[i] / sqrtf(piv[i]) : 0.0f;
+  for (int i = 0; i < NB; ++i) LiT[lane][i] = (i >= lane) ? rr[i] * rsm[i] : 0.0f;
   __syncwarp();
 }
 
@@ -186,7 +227,7 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
   __shared__ __align__(16) float S2[NB][TS];
   __shared__ __align__(16) float S3[NB][TS];
   __shared__ __align__(16) float S4[NB][TS];
-  __shared__ float colv[2 * NB];
+  __shared__ __align__(16) float colv[3 * NB];  // two pivot-column buffers + 1/sqrt(pivot)
   const int tid = threadIdx.x;
   const int ty = tid >> 3, tx = tid & 7;
   const int d = a.d, D = a.D;
@@ -242,11 +283,15 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
       if (it < n_panel) {
         // ------------------------------------------------ panel item
         const int r = j + it;
-        load_nat(S0, P, d, j, j, true);  // diagonal block
-        if (r > j) load_nat(S1, P, d, r, j, false);
-        if (j > 0) {
-          load_tr(S2, P, d, j, j - 1);  // L(j, j-1)^T
-          if (r > j) load_tr(S3, P, d, r, j - 1);
+        {
+          const TileRegs t0 = fetch(P, d, j, j, true);                    // diagonal block
+          const TileRegs t1 = fetch(P, d, r > j ? r : D, j);              // own block (none when r == j)
+          const TileRegs t2 = fetch(P, d, j > 0 ? j : D, j - 1);          // L(j, j-1)
+          const TileRegs t3 = fetch(P, d, (j > 0 && r > j) ? r : D, j - 1);  // L(r, j-1)
+          put_nat(S0, t0);
+          put_nat(S1, t1);
+          put_tr(S2, t2);
+          put_tr(S3, t3);
         }
         __syncthreads();
         if (j > 0) {
@@ -263,12 +308,12 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
               if (r > j) S1[2 * ty + p][4 * tx + q] -= acc2[p][q];
             }
         }
-        __syncthreads();
-        if (tid < 32) warp_factor_invert(S0, S4, colv, d, j * NB, a.status);
         // S3 <- tile(r, j) transposed, for the triangular solve
         if (r > j) {
           for (int e = tid; e < NB * NB; e += kThreads) S3[e & 31][e >> 5] = S1[e >> 5][e & 31];
         }
+        __syncthreads();
+        if (tid < 32) warp_factor_invert(S0, S4, colv, colv + 2 * NB, d, j * NB, a.status);
         __syncthreads();
         if (r == j) {
           float* out = a.side + (size_t)j * NB * NB;  // natural layout: out[y][m] = S4[m][y]
@@ -292,8 +337,20 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
         while (rr * (rr + 1) / 2 > t) --rr;
         const int cc = t - rr * (rr + 1) / 2;
         const int r = j + 1 + rr, c = j + 1 + cc;
-        load_tr(S0, P, d, r, j - 1);
-        load_tr(S1, P, d, c, j - 1);
+        float old[2][4];
+        {
+          const TileRegs t0 = fetch(P, d, r, j - 1);
+          const TileRegs t1 = fetch(P, d, c, j - 1);
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int gr = r * NB + 2 * ty + p, gc = c * NB + 4 * tx + q;
+              old[p][q] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : 0.0f;
+            }
+          put_tr(S0, t0);
+          put_tr(S1, t1);
+        }
         __syncthreads();
         zero(acc);
         mma32(acc, S0, S1, ty, tx);
@@ -302,18 +359,19 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int gr = r * NB + 2 * ty + p, gc = c * NB + 4 * tx + q;
-            if (gr < d && gc < d) {
-              float* dst = P + (size_t)gr * d + gc;
-              *dst = ldp(dst) - acc[p][q];
-            }
+            if (gr < d && gc < d) P[(size_t)gr * d + gc] = old[p][q] - acc[p][q];
           }
       } else {
         // ------------------------------------------------ inverse item: column block c, rows chunk
         const int t = it - n_panel - n_trail;
         const int c = t / per_c, ch = t % per_c;
         // Y(j-1, c) = Linv_{j-1} R(j-1, c);  R(j-1, j-1) = I, else R(j-1, c) sits transposed at P(c, j-1)
-        load_tr_block(S0, a.side + (size_t)(j - 1) * NB * NB);  // S0[m][x] = Linv[x][m]
-        if (c < j - 1) load_tr(S1, P, d, c, j - 1);            // S1[m][y] = R(j-1, c)[m][y]
+        {
+          const TileRegs t0 = fetch_block(a.side + (size_t)(j - 1) * NB * NB);
+          const TileRegs t1 = fetch(P, d, c < j - 1 ? c : D, j - 1);
+          put_tr(S0, t0);  // S0[m][x] = Linv[x][m]
+          put_tr(S1, t1);  // S1[m][y] = R(j-1, c)[m][y]  (R(j-1, c) is stored transposed at P(c, j-1))
+        }
         __syncthreads();
         if (c < j - 1) {
           zero(acc);
@@ -340,22 +398,26 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
         const int i0 = j + ch * kYChunk;
         const int i1 = min(i0 + kYChunk, D);
         for (int i = i0; i < i1; ++i) {
+          float old[2][4];
+          const TileRegs t3 = fetch(P, d, i, j - 1);
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {  // R(i, c) is stored transposed at P(c, i)
+              const int gr = c * NB + 4 * tx + q, gc = i * NB + 2 * ty + p;
+              old[p][q] = (gr < d && gc < d) ? ldp(P + (size_t)gr * d + gc) : 0.0f;
+            }
           __syncthreads();
-          load_tr(S3, P, d, i, j - 1);  // S3[m][x] = L(i, j-1)[x][m]
+          put_tr(S3, t3);  // S3[m][x] = L(i, j-1)[x][m]
           __syncthreads();
           zero(acc);
           mma32(acc, S3, S2, ty, tx);
-          // R(i, c) is stored transposed at P(c, i)
 #pragma unroll
           for (int p = 0; p < 2; ++p)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const int x = 2 * ty + p, y = 4 * tx + q;
-              const int gr = c * NB + y, gc = i * NB + x;
-              if (gr < d && gc < d) {
-                float* dst = P + (size_t)gr * d + gc;
-                *dst = ldp(dst) - acc[p][q];
-              }
+              const int gr = c * NB + 4 * tx + q, gc = i * NB + 2 * ty + p;
+              if (gr < d && gc < d) P[(size_t)gr * d + gc] = old[p][q] - acc[p][q];
             }
         }
       }
@@ -381,7 +443,7 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
   }
 }
 
-constexpr size_t kSideOffset = 256;
+constexpr size_t kSideOffset = 1024;
 
 }  // namespace
 
@@ -398,8 +460,8 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
   a.H = H;
   a.P = U;
   a.lam = reinterpret_cast<float*>(ws);
-  a.bar = reinterpret_cast<unsigned*>(ws + 64);
-  a.abort_flag = reinterpret_cast<int*>(ws + 128);
+  a.bar = reinterpret_cast<unsigned*>(ws + 256);
+  a.abort_flag = reinterpret_cast<int*>(ws + 512);
   a.side = reinterpret_cast<float*>(ws + kSideOffset);
   a.status = status;
   a.damp = damp;
@@ -412,9 +474,9 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
   if (!coop) return GPTQ_ERR_CUDA;
   GPTQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prepare_kernel, kThreads, 0));
   if (occ < 1) return GPTQ_ERR_CUDA;
-  const int grid = sms * (occ < 2 ? occ : 2);
+  const int grid = sms;  // one CTA per SM: enough items per phase for the sizes this path serves
   GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), stream));
-  GPTQ_CUDA_TRY(cudaMemsetAsync(ws + 64, 0, 128, stream));  // barrier words and abort flag
+  GPTQ_CUDA_TRY(cudaMemsetAsync(ws + 256, 0, 512, stream));  // barrier words and abort flag
   void* args[] = {&a};
   GPTQ_CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(prepare_kernel), dim3(grid), dim3(kThreads),
                                             args, 0, stream));

@@ -39,69 +39,84 @@ __global__ void __launch_bounds__(256) convert_rowgrid_kernel(const T* __restric
     mn = warp_min(mn);
     mx = warp_max(mx);
     if (lane == 0) {
-      float s, z;
-      grid_from_range(mn, mx, (float)((1 << bits) - 1), s, z);
+      float s, z, rs;
+      grid_from_range(mn, mx, (float)((1 << bits) - 1), s, z, rs);
       scales[row] = s;
       zeros[row] = (int32_t)z;
     }
   }
 }
 
-// Column loop of one row over block [i1, i1 + 32*NS), run by one warp.  v[s] holds column
-// i1 + 32*s + lane of the row (current values).  Us is the block's corner of U (strict upper part,
-// row-major B x B) and invd the reciprocals of its diagonal.  Each step broadcasts w_i from its
-// lane, rounds it, and applies err_i * U[i, j] to the columns of the block.  The inner loop is not
-// unrolled: one copy of the step per register slot keeps the code small enough for the i-cache.
+// Column loop of one row over block [i1, i1 + 32*NS), run by one warp.  Lane L holds the NS
+// consecutive columns i1 + NS*L .. i1 + NS*L + NS-1 in v[0..NS-1] (current values).  Us is the
+// block's corner of U (strict upper part, row-major B x B) and invd the reciprocals of its diagonal.
+//
+// Step i (owner lane L = i / NS, slot s = i % NS): every lane rounds its own v[s] (only the owner's
+// result is kept), the owner's error is broadcast, and every lane applies err * U[i, j] to its
+// columns.  The owner updates its next column from its own error before the broadcast lands, so the
+// dependency chain leaves the lane only once every NS steps.
 template <int NS>
 __device__ __forceinline__ void column_loop(float (&v)[NS], const float* __restrict__ Us,
                                             const float* __restrict__ invd, int i1, int group_size,
                                             int n_groups, float maxq, float& scale, float& zero,
-                                            const float* wrow, int64_t row, float* __restrict__ scales,
-                                            int32_t* __restrict__ zeros, uint32_t (&code_reg)[NS],
-                                            float (&err_reg)[NS]) {
+                                            float& rscale, const float* wrow, int64_t row,
+                                            float* __restrict__ scales, int32_t* __restrict__ zeros,
+                                            uint32_t (&code_reg)[NS], float (&err_reg)[NS]) {
   constexpr int B = 32 * NS;
   const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int s = 0; s < NS; ++s) {
 #pragma unroll 1
-    for (int l = 0; l < 32; ++l) {
-      const int i = s * 32 + l;
-      if (group_size != 0 && l == 0 && ((i1 + i) % group_size) == 0) {
+  for (int L = 0; L < 32; ++L) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const int i = L * NS + s;
+      if (group_size != 0 && s == 0 && ((i1 + i) % group_size) == 0) {
         // grid of the group starting here, from the current values of its columns
-        const int gw = group_size / 32;  // register slots the group covers inside the block
+        const int c_end = i + group_size;  // block-local end (may pass the block)
         float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < NS; ++t)
-          if (t >= s && t < s + gw) {
+        for (int t = 0; t < NS; ++t) {
+          const int c = lane * NS + t;
+          if (c >= i && c < c_end) {
             mn = fminf(mn, v[t]);
             mx = fmaxf(mx, v[t]);
           }
-        for (int c = i1 + B + lane; c < i1 + i + group_size; c += 32) {  // group wider than the block
+        }
+        for (int c = i1 + B + lane; c < i1 + c_end; c += 32) {  // group wider than the block
           const float x = wrow[c];
           mn = fminf(mn, x);
           mx = fmaxf(mx, x);
         }
         mn = warp_min(mn);
         mx = warp_max(mx);
-        grid_from_range(mn, mx, maxq, scale, zero);
+        grid_from_range(mn, mx, maxq, scale, zero, rscale);
         if (lane == 0) {
           const int g = (i1 + i) / group_size;
           scales[row * n_groups + g] = scale;
           zeros[row * n_groups + g] = (int32_t)zero;
         }
       }
-      const float wi = __shfl_sync(0xffffffffu, v[s], l);
-      float q = rintf(__fdiv_rn(wi, scale)) + zero;
-      q = fminf(fmaxf(q, 0.0f), maxq);
-      const float deq = scale * (q - zero);
-      const float err = (wi - deq) * invd[i];
-      if (lane == l) {
-        code_reg[s] = (uint32_t)q;
+      const bool owner = (lane == L);
+      const float wi = owner ? v[s] : 0.0f;  // only the owner's value matters
+      // code - zero, clamped to the grid; the quotient as an IEEE fp32 product with 1/scale
+      const float qz = fminf(fmaxf(rintf(__fmul_rn(wi, rscale)), -zero), maxq - zero);
+      const float delta = fmaf(-scale, qz, wi);  // w_i - dequantized value
+      const float err = delta * invd[i];
+      if (owner) {
+        code_reg[s] = (uint32_t)(qz + zero);
         err_reg[s] = err;
       }
-      const float* urow = Us + i * B;
+      // Us rows are pre-divided by U_ii: err * U[i][j] = delta * Us[i][j]
+      const float* urow = Us + i * B + lane * NS;
+      if (s + 1 < NS && owner) v[s + 1] = fmaf(-delta, urow[s + 1], v[s + 1]);  // owner's next column first
+      const float e = __shfl_sync(0xffffffffu, delta, L);
 #pragma unroll
-      for (int t = 0; t < NS; ++t) v[t] = fmaf(-err, urow[t * 32 + lane], v[t]);
+      for (int t = 0; t < NS; ++t) {
+        if (t == s + 1) {
+          if (!owner) v[t] = fmaf(-e, urow[t], v[t]);
+        } else {
+          v[t] = fmaf(-e, urow[t], v[t]);
+        }
+      }
     }
   }
 }
@@ -122,14 +137,33 @@ __device__ __forceinline__ void grid_at_block(int64_t row, int i1, int group_siz
   }
 }
 
-// Loads U[i1:i1+B, i1:i1+B] (strict upper part) and the reciprocals of its diagonal.
+// Loads the block's corner of U, strict upper part, each row divided by its diagonal entry
+// (Us[r][c] = U[i1+r][i1+c] / U[i1+r][i1+r]), and the reciprocals of the diagonal.  All of a thread's
+// float4 loads are issued before the first store (one L2 round trip per call).
 template <int B>
 __device__ __forceinline__ void load_u_block(float* Us, float* invd, const float* __restrict__ U, int d, int i1) {
-  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
-    const int r = e / B, c = e % B;
-    Us[e] = (c > r) ? U[(size_t)(i1 + r) * d + i1 + c] : 0.0f;
+  constexpr int PER = B * B / 4 / 256;  // float4 per thread (blockDim.x == 256)
+  float4 v[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int e = threadIdx.x + 256 * k;
+    const int r = e / (B / 4), c = (e % (B / 4)) * 4;
+    v[k] = *reinterpret_cast<const float4*>(U + (size_t)(i1 + r) * d + i1 + c);
   }
-  for (int r = threadIdx.x; r < B; r += blockDim.x) invd[r] = 1.0f / U[(size_t)(i1 + r) * d + i1 + r];
+  if (threadIdx.x < B) invd[threadIdx.x] = 1.0f / U[(size_t)(i1 + threadIdx.x) * d + i1 + threadIdx.x];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int e = threadIdx.x + 256 * k;
+    const int r = e / (B / 4), c = (e % (B / 4)) * 4;
+    const float ir = invd[r];
+    float4 u = v[k];
+    u.x = (c + 0 > r) ? u.x * ir : 0.0f;
+    u.y = (c + 1 > r) ? u.y * ir : 0.0f;
+    u.z = (c + 2 > r) ? u.z * ir : 0.0f;
+    u.w = (c + 3 > r) ? u.w * ir : 0.0f;
+    *reinterpret_cast<float4*>(Us + r * B + c) = u;
+  }
 }
 
 // Column loop over block [i1, i1 + 32*NS) for 8 rows per CTA (per-block launch path).
@@ -152,19 +186,20 @@ __global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int
   float* wr = w + row * d;
   float v[NS];
 #pragma unroll
-  for (int s = 0; s < NS; ++s) v[s] = wr[i1 + s * 32 + lane];
+  for (int s = 0; s < NS; ++s) v[s] = wr[i1 + lane * NS + s];
   const float maxq = (float)((1 << bits) - 1);
   const int n_groups = group_size ? d / group_size : 1;
   float scale, zero;
   grid_at_block(row, i1, group_size, n_groups, scales, zeros, scale, zero);
+  float rscale = __frcp_rn(scale);
   uint32_t code_reg[NS];
   float err_reg[NS];
-  column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, wr, row, scales, zeros, code_reg,
-                  err_reg);
+  column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, rscale, wr, row, scales, zeros,
+                  code_reg, err_reg);
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
-    codes[row * d + i1 + s * 32 + lane] = (uint8_t)code_reg[s];
-    err_out[row * B + s * 32 + lane] = err_reg[s];
+    codes[row * d + i1 + lane * NS + s] = (uint8_t)code_reg[s];
+    err_out[row * B + lane * NS + s] = err_reg[s];
   }
 }
 
@@ -204,14 +239,14 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
       mn = warp_min(mn);
       mx = warp_max(mx);
       if (lane == 0) {
-        float s, z;
-        grid_from_range(mn, mx, maxq, s, z);
+        float s, z, rs;
+        grid_from_range(mn, mx, maxq, s, z, rs);
         scales[row] = s;
         zeros[row] = (int32_t)z;
       }
     }
   }
-  float scale = 1.0f, zero = 0.0f;
+  float scale = 1.0f, zero = 0.0f, rscale = 1.0f;
   for (int i1 = 0; i1 < d; i1 += B) {
     __syncthreads();
     load_u_block<B>(Us, invd, U, d, i1);
@@ -220,31 +255,49 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
       __syncwarp();
       if (i1 == 0 || group_size == 0) {
         grid_at_block(row, i1, group_size, n_groups, scales, zeros, scale, zero);
+        rscale = __frcp_rn(scale);
       }
       float v[NS];
 #pragma unroll
-      for (int s = 0; s < NS; ++s) v[s] = wr[i1 + s * 32 + lane];
+      for (int s = 0; s < NS; ++s) v[s] = wr[i1 + lane * NS + s];
       uint32_t code_reg[NS];
       float err_reg[NS];
-      column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, wr, row, scales, zeros,
-                      code_reg, err_reg);
+      column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, rscale, wr, row, scales,
+                      zeros, code_reg, err_reg);
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        codes[row * d + i1 + s * 32 + lane] = (uint8_t)code_reg[s];
-        errs[warp * B + s * 32 + lane] = err_reg[s];
+        codes[row * d + i1 + lane * NS + s] = (uint8_t)code_reg[s];
+        errs[warp * B + lane * NS + s] = err_reg[s];
       }
     }
-    // lazy update of this CTA's rows over the columns after the block
+    // lazy update of this CTA's rows over the columns after the block; the next chunk of the U
+    // panel is loaded into registers while the current one is used from shared memory
+    constexpr int PER = B * CW / 4 / 256;  // float4 of a chunk per thread
+    float4 uv[PER];
+    auto fetch_chunk = [&](int c0) {
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int e = threadIdx.x + 256 * k;
+        const int r = e / (CW / 4), c = (e % (CW / 4)) * 4;
+        uv[k] = (c0 + c < d) ? *reinterpret_cast<const float4*>(U + (size_t)(i1 + r) * d + c0 + c)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    if (i1 + B < d) fetch_chunk(i1 + B);
     for (int c0 = i1 + B; c0 < d; c0 += CW) {
+      const bool mine = valid && c0 + 4 * lane < d;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (mine) o = *reinterpret_cast<const float4*>(wr + c0 + 4 * lane);
       __syncthreads();
-      for (int e = threadIdx.x; e < B * CW / 4; e += blockDim.x) {
-        const int k = e / (CW / 4), c = (e % (CW / 4)) * 4;
-        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c0 + c < d) u = *reinterpret_cast<const float4*>(U + (size_t)(i1 + k) * d + c0 + c);
-        *reinterpret_cast<float4*>(Us + k * CW + c) = u;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int e = threadIdx.x + 256 * k;
+        const int r = e / (CW / 4), c = (e % (CW / 4)) * 4;
+        *reinterpret_cast<float4*>(Us + r * CW + c) = uv[k];
       }
       __syncthreads();
-      if (valid && c0 + 4 * lane < d) {
+      if (c0 + CW < d) fetch_chunk(c0 + CW);
+      if (mine) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         const float* er = errs + warp * B;
 #pragma unroll 8
@@ -256,13 +309,11 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
           acc.z = fmaf(e, u.z, acc.z);
           acc.w = fmaf(e, u.w, acc.w);
         }
-        float4* dst = reinterpret_cast<float4*>(wr + c0 + 4 * lane);
-        float4 o = *dst;
         o.x -= acc.x;
         o.y -= acc.y;
         o.z -= acc.z;
         o.w -= acc.w;
-        *dst = o;
+        *reinterpret_cast<float4*>(wr + c0 + 4 * lane) = o;
       }
     }
   }
