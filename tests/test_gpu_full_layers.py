@@ -1,0 +1,128 @@
+"""GPU parity at the full sizes of the large layers (the launch configurations bench.py times).
+
+The oracle cannot afford an fp64 H of every large layer end to end, so each stage is checked on
+what it can compute exactly, and no stage takes an input from the CUDA path:
+
+* H: the full GPU Hessian against fp64 on sampled 128x128 blocks (diagonal, off-diagonal and
+  outlier-channel blocks), all 262,144 tokens.
+* U: the trailing k x k principal block of U depends only on the trailing k x k block of the
+  dampened Hessian (write Hd = R R^T with R upper: U = R^-1 and U_22 = R_22^-1).  The oracle builds
+  that block (and the damping from all column norms) from X in fp64 and factors it.
+* Column loop: the full m x d layer quantized on the GPU with an oracle U (from a token subsample
+  of the same inputs) against the oracle's quantization of the same rows with the same U.
+* End to end on the 4096-wide layer: all stages chained on the GPU against the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_21_b200 import workloads as wl
+
+import gpu_support as S
+
+pytestmark = pytest.mark.gpu
+
+LARGE = ["llama7b_q_4096x4096", "llama7b_up_11008x4096", "llama7b_down_4096x11008"]
+
+
+def _blocks(d, oc, rng):
+    starts = sorted({0, d - 128, (d // 2) // 128 * 128} | {int(c) // 128 * 128 for c in oc[:3]})
+    pairs = [(a, a) for a in starts] + [(starts[0], starts[-1]), (starts[1], starts[-1])]
+    pairs += [(int(rng.integers(0, d // 128)) * 128, int(rng.integers(0, d // 128)) * 128) for _ in range(4)]
+    return [(min(a, b), max(a, b)) for a, b in pairs]
+
+
+def _x_cpu_chunks(X, step=16384):
+    for t0 in range(0, X.shape[0], step):
+        yield X[t0:t0 + step].cpu().double().numpy()
+
+
+@pytest.mark.parametrize("name", ["llama7b_q_4096x4096", "llama7b_down_4096x11008"])
+def test_hessian_sampled_blocks(name):
+    L = wl.LAYERS[name]
+    X = wl.make_x(L, device="cuda")
+    H = S.hessian(X)
+    rng = np.random.default_rng(0)
+    blocks = _blocks(L.d, wl.outlier_channels(L).numpy(), rng)
+    ref = {p: np.zeros((128, 128)) for p in blocks}
+    for Xc in _x_cpu_chunks(X):
+        for (a, b) in blocks:
+            ref[(a, b)] += 2.0 * Xc[:, a:a + 128].T @ Xc[:, b:b + 128]
+    num = den = 0.0
+    for (a, b), R in ref.items():
+        G = H[a:a + 128, b:b + 128].double().cpu().numpy()
+        if a == b:
+            iu = np.triu_indices(128)
+            G, R = G[iu], R[iu]
+        num += np.sum((G - R) ** 2)
+        den += np.sum(R ** 2)
+    assert np.sqrt(num / den) <= S.H_REL_FRO
+
+
+@pytest.mark.parametrize("name", ["llama7b_q_4096x4096", "llama7b_down_4096x11008"])
+def test_prepare_trailing_block(name):
+    L = wl.LAYERS[name]
+    k = 512
+    X = wl.make_x(L, device="cuda")
+    H = S.hessian(X)
+    U = S.prepare(H, L.damp)[-k:, -k:].double().cpu().numpy()
+    colsq = np.zeros(L.d)
+    Hk = np.zeros((k, k))
+    for Xc in _x_cpu_chunks(X):
+        colsq += np.einsum("ij,ij->j", Xc, Xc)
+        Hk += 2.0 * Xc[:, -k:].T @ Xc[:, -k:]
+    lam = L.damp * np.mean(2.0 * colsq)
+    Hd_k = Hk + lam * np.eye(k)
+    Uref = oracle.inverse_upper_cholesky(Hd_k)
+    rel = np.linalg.norm(U - Uref) / np.linalg.norm(Uref)
+    kappa = np.linalg.cond(Hd_k)
+    assert rel <= max(1e-5, 10 * kappa * 6e-8), (rel, kappa)
+    assert np.all(U[np.tril_indices(k, -1)] == 0.0)
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_quantize_full_layer_with_oracle_u(name):
+    L = wl.LAYERS[name]
+    Lsub = L.with_tokens(8 * 2048)
+    Xs = wl.make_x(Lsub).double().numpy()
+    Hs = oracle.hessian(Xs)
+    U = oracle.inverse_upper_cholesky(oracle.dampen(Hs, L.damp))
+    U32 = np.ascontiguousarray(U, dtype=np.float32)
+    W = wl.make_w(L)
+    gpu = S.quantize(W.cuda(), torch.from_numpy(U32).cuda(), L.bits, L.group_size, L.block_size)
+    rows = np.sort(np.random.default_rng(1).choice(L.m, size=min(L.m, 512), replace=False))
+    ref = oracle.gptq_quantize(W[rows].double().numpy(), U32.astype(np.float64), L.bits, L.group_size,
+                               L.block_size)
+    Wr = W[rows].double().numpy()
+    st = S.compare_quantization((gpu[0][rows], gpu[1][rows], gpu[2][rows]), ref, L.group_size, Wr, Hs,
+                                label=name)
+    print(name, st)
+
+
+def test_end_to_end_llama_q_layer():
+    L = wl.LAYERS["llama7b_q_4096x4096"]
+    X = wl.make_x(L, device="cuda")
+    W = wl.make_w(L)
+    from post_weight_quantization_21_b200 import LayerSolver
+    s = LayerSolver(L.m, L.d, L.n_tokens, L.bits, L.group_size, L.block_size, L.damp, X.dtype, W.dtype)
+    s.X.copy_(X)
+    s.W.copy_(W)
+    s.run()
+    s.check_status()
+    torch.cuda.synchronize()
+    H = np.zeros((L.d, L.d))
+    for Xc in _x_cpu_chunks(X):
+        oracle.hessian_accumulate(H, Xc)
+    del X
+    rows = np.sort(np.random.default_rng(2).choice(L.m, size=1024, replace=False))
+    U = oracle.inverse_upper_cholesky(oracle.dampen(H, L.damp))
+    Wr = W[rows].double().numpy()
+    ref = oracle.gptq_quantize(Wr, U, L.bits, L.group_size, L.block_size)
+    ref["E"] = oracle.reconstruction_error(Wr, ref["Wq"], H)
+    gpu = (s.codes.cpu().numpy().astype(np.int64)[rows], s.scales.cpu().numpy()[rows],
+           s.zeros.cpu().numpy().astype(np.int64)[rows])
+    st = S.compare_quantization(gpu, ref, L.group_size, Wr, H, ref["E"], label=L.name)
+    packed = s.packed.cpu().numpy()[rows]
+    np.testing.assert_array_equal(packed, oracle.pack_codes(gpu[0], L.bits))
+    print("llama q end-to-end", st)
