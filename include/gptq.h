@@ -112,6 +112,27 @@ GPTQ_API gptq_status gptq_prepare_uinv(const float* H, int64_t d, float damp, fl
 GPTQ_API size_t gptq_prepare_workspace_size(int64_t d);
 
 /* ------------------------------------------------------------------------------------------
+ * gptq_prepare_uinv_static: the same computation as gptq_prepare_uinv without a workspace argument.
+ *
+ * The GPTQ pages have no counterpart for this call; it exists for callers that cannot allocate
+ * device memory themselves, for example a plugin whose host application owns all device memory
+ * through its own pool, or a latency-bound path where no allocator may be called.  The scratch the
+ * computation needs (about 1 MiB) is a fixed array compiled into this library; every GPU that loads
+ * the library holds it until the process exits.
+ *
+ *   H, d, damp, U, dev_status, stream: as for gptq_prepare_uinv (U is still caller memory).
+ *   d > GPTQ_PREPARE_STATIC_MAX_D returns GPTQ_ERR_WORKSPACE and enqueues nothing.
+ *   The first call on each device looks up the array's device address (a host-side runtime call,
+ *   with that device current); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents (each call clears the parts
+ *   that must start at zero).  Calls that overlap on the GPU, on any streams, race on it: order them.
+ *   No memory is allocated or freed.
+ * ------------------------------------------------------------------------------------------ */
+#define GPTQ_PREPARE_STATIC_MAX_D 8192
+GPTQ_API gptq_status gptq_prepare_uinv_static(const float* H, int64_t d, float damp, float* U,
+                                              int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * A4 - A6  Column loop with error compensation and lazy block updates.
  *
  * For each column i in natural order (FDE breakdown figure steps 1-4): q_i = clamp(rint(w_i/scale)

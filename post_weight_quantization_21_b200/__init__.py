@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "GPTQError", "lib", "gptq_hessian_accumulate", "gptq_hessian_workspace_size", "gptq_prepare_uinv",
-    "gptq_prepare_workspace_size", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
+    "gptq_prepare_workspace_size", "gptq_prepare_uinv_static", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
     "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
 ]
 
@@ -46,6 +46,7 @@ ABI_FUNCTIONS = {
     "gptq_hessian_workspace_size": (_sz, [_i64, _i64, _i32]),
     "gptq_prepare_uinv": (_i32, [_vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "gptq_prepare_workspace_size": (_sz, [_i64]),
+    "gptq_prepare_uinv_static": (_i32, [_vp, _i64, _f32, _vp, _vp, _vp]),
     "gptq_quantize_layer": (_i32, [_vp, _i32, _i64, _i64, _vp, ctypes.POINTER(QuantCfg), _vp, _vp, _vp,
                                    _vp, _sz, _vp]),
     "gptq_quantize_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
@@ -139,6 +140,18 @@ def gptq_prepare_uinv(H: torch.Tensor, U: torch.Tensor, status: torch.Tensor, wo
     st = lib().gptq_prepare_uinv(_ptr(H), H.shape[0], damp, _ptr(U), _ptr(status), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "gptq_prepare_uinv")
+
+
+PREPARE_STATIC_MAX_D = 8192
+
+
+def gptq_prepare_uinv_static(H: torch.Tensor, U: torch.Tensor, status: torch.Tensor, damp: float = 0.01,
+                             stream=None):
+    """gptq_prepare_uinv without a workspace, for callers that cannot allocate: the library's own
+    fixed scratch array (d <= PREPARE_STATIC_MAX_D) is used.  Calls overlapping on the GPU race."""
+    _contig(H, "H"), _contig(U, "U")
+    st = lib().gptq_prepare_uinv_static(_ptr(H), H.shape[0], damp, _ptr(U), _ptr(status), _stream(stream))
+    _check(st, "gptq_prepare_uinv_static")
 
 
 # ------------------------------------------------------------------------------------------ A4 - A6

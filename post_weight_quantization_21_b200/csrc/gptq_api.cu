@@ -95,6 +95,15 @@ gptq_status gptq_prepare_uinv(const float* H, int64_t d, float damp, float* U, i
   return gptq::prepare_launch(H, d, damp, U, dev_status, workspace, static_cast<cudaStream_t>(stream));
 }
 
+gptq_status gptq_prepare_uinv_static(const float* H, int64_t d, float damp, float* U, int32_t* dev_status,
+                                     void* stream) {
+  if (d <= 0 || H == nullptr || U == nullptr || dev_status == nullptr) return GPTQ_ERR_ARG;
+  if (!(damp >= 0.0f) || !aligned(H, 16) || !aligned(U, 16) || !aligned(dev_status, 4)) return GPTQ_ERR_ARG;
+  if ((const void*)H == (const void*)U) return GPTQ_ERR_ARG;
+  if (d > GPTQ_PREPARE_STATIC_MAX_D) return GPTQ_ERR_WORKSPACE;
+  return gptq::prepare_launch_static(H, d, damp, U, dev_status, static_cast<cudaStream_t>(stream));
+}
+
 size_t gptq_quantize_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* cfg) {
   if (m <= 0 || d <= 0 || d > kMaxDim || m > kMaxDim * 64 || cfg == nullptr) return 0;
   if (check_cfg(cfg, d) != GPTQ_OK) return 0;

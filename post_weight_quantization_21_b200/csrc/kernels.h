@@ -25,6 +25,9 @@ gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, 
 size_t prepare_workspace(int64_t d);
 gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
                            void* workspace, cudaStream_t stream);
+// same, with the scratch in a static device array (d <= GPTQ_PREPARE_STATIC_MAX_D)
+gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* U, int32_t* status,
+                                  cudaStream_t stream);
 
 // A4 - A6
 size_t quantize_workspace(int64_t m, int64_t d, int block_size);

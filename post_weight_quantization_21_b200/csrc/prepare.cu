@@ -26,6 +26,8 @@
 //   phase R   U = J Y J: lower block triangle -> upper, strict lower part zeroed.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -482,6 +484,50 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
                                             args, 0, stream));
   count_launch();
   return GPTQ_OK;
+}
+
+}  // namespace gptq
+
+namespace gptq {
+// ------------------------------------------------------------------------------------------------
+// Allocation-free variant.  The prepare kernel's scratch (damping value, barrier words, the inverse
+// diagonal blocks: 1 KiB + d/32 * 4 KiB) lives in this file-scope device array instead of a caller
+// workspace, sized for d <= GPTQ_PREPARE_STATIC_MAX_D.  Every GPU that loads the library keeps it for
+// the life of the process.
+namespace {
+constexpr size_t kStaticScratchBytes =
+    kSideOffset + (size_t)(GPTQ_PREPARE_STATIC_MAX_D / NB) * NB * NB * sizeof(float);
+static __device__ __align__(256) unsigned char g_prepare_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_address[kMaxDevices] = {};
+
+// Device address of g_prepare_scratch on the current device; looked up once per device, with that
+// device current.  Host code must not use the symbol itself: it is a host-side stand-in.
+gptq_status static_scratch(void** out) {
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return GPTQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_address[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_prepare_scratch) != cudaSuccess || p == nullptr) return GPTQ_ERR_CUDA;
+    g_scratch_address[dev] = p;
+  }
+  *out = g_scratch_address[dev];
+  return GPTQ_OK;
+}
+}  // namespace
+
+gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* U, int32_t* status,
+                                  cudaStream_t stream) {
+  static_assert(kStaticScratchBytes >= kSideOffset + 256 * NB * NB * sizeof(float), "scratch too small");
+  void* scratch = nullptr;
+  gptq_status st = static_scratch(&scratch);
+  if (st != GPTQ_OK) return st;
+  if (prepare_workspace(d) > kStaticScratchBytes) return GPTQ_ERR_WORKSPACE;
+  return prepare_launch(H, d, damp, U, status, scratch, stream);
 }
 
 }  // namespace gptq
