@@ -96,14 +96,20 @@ def compare_quantization(gpu, ref, group_size, W=None, H=None, E_ref=None, label
         assert np.array_equal(zeros, rz), f"{label}: zeros differ"
         checked = m
     else:
-        # per-group grids depend on the row's earlier codes: check the (row, group) pairs up to and
-        # including the group of the row's first mismatch; later ones are counted
+        # per-group grids depend on the row's earlier codes.  Groups before the row's first mismatch
+        # must match (scales within tolerance, zeros equal); in the group of the first mismatch the
+        # scale must match and the zero point may sit one level off (its rounding is a near-tie of
+        # the same kind as a code's); later groups follow a different trajectory and are counted.
         ng = d // group_size
-        ok = (np.arange(ng)[None, :] * group_size) <= first_bad[:, None]
+        gstart = np.arange(ng)[None, :] * group_size
+        before = gstart + group_size <= first_bad[:, None]
+        at = (gstart <= first_bad[:, None]) & ~before
         rel = np.abs(scales - rs) / np.abs(rs)
-        assert rel[ok].max() <= SCALE_REL, f"{label}: group scale rel err {rel[ok].max()}"
-        assert np.array_equal(zeros[ok], rz[ok]), f"{label}: group zeros differ"
-        checked = int(ok.sum())
+        upto = before | at
+        assert rel[upto].max() <= SCALE_REL, f"{label}: group scale rel err {rel[upto].max()}"
+        assert np.array_equal(zeros[before], rz[before]), f"{label}: group zeros differ"
+        assert np.all(np.abs(zeros[at] - rz[at]) <= 1), f"{label}: zero point off by more than one"
+        checked = int(upto.sum())
     stats = {"agree": agree, "mismatches": int(np.sum(diff != 0)), "rows_diverged": int(bad_rows.sum()),
              "max_level_diff": int(np.abs(diff).max()), "grids_checked": checked}
     if W is not None and H is not None:
