@@ -31,7 +31,7 @@ gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* 
 
 // A4 - A6
 size_t quantize_workspace(int64_t m, int64_t d, int block_size);
-bool quantize_fused(int64_t d);  // one launch per layer (U resident in L2) rather than launches per block
+bool quantize_fused(int64_t m, int64_t d);  // one launch per layer (U resident in L2) rather than launches per block
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
                             void* workspace, cudaStream_t stream);

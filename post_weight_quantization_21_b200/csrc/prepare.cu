@@ -476,7 +476,10 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
   if (!coop) return GPTQ_ERR_CUDA;
   GPTQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prepare_kernel, kThreads, 0));
   if (occ < 1) return GPTQ_ERR_CUDA;
-  const int grid = sms;  // one CTA per SM: enough items per phase for the sizes this path serves
+  // One CTA per SM.  (Two co-resident CTAs per SM gave wrong, run-to-run different results at
+  // d >= 512 although every item of a phase touches disjoint tiles; until that is understood the
+  // launch keeps one CTA per SM, which is exact and bit-reproducible.)
+  const int grid = sms;
   GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), stream));
   GPTQ_CUDA_TRY(cudaMemsetAsync(ws + 256, 0, 512, stream));  // barrier words and abort flag
   void* args[] = {&a};

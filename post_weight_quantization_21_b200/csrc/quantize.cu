@@ -319,50 +319,96 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
   }
 }
 
-// w[:, i2:] -= Err[:, 0:B] * U[i1:i1+B, i2:]; 64x64 output tile per CTA, K = B in steps of 32.
+// w[:, i2:] -= Err[:, 0:B] * U[i1:i1+B, i2:] (lazy update of all rows for one block).
+// 128x128 output tile per CTA, 256 threads with 8x8 outputs each (rows ty*4+{0..3} and 64+ty*4+{0..3},
+// likewise columns), K = B staged 32 at a time through shared memory; the next K slice is loaded
+// into registers while the current one is used.
 template <int B>
-__global__ void __launch_bounds__(256) lazy_update_kernel(float* __restrict__ w, int64_t m, int d, int i1,
-                                                          const float* __restrict__ U,
-                                                          const float* __restrict__ err) {
-  constexpr int KC = 32;
-  __shared__ __align__(16) float Et[KC][64 + 4];  // Et[k][row]
-  __shared__ __align__(16) float Ut[KC][64 + 4];  // Ut[k][col]
+__global__ void __launch_bounds__(256) lazy_gemm_kernel(float* __restrict__ w, int64_t m, int d, int i1,
+                                                        const float* __restrict__ U,
+                                                        const float* __restrict__ err) {
+  constexpr int KC = 32, TM = 128, TN = 128, LDA = TM + 4, LDB = TN + 4;
+  __shared__ __align__(16) float As[KC][LDA];  // As[k][row] = err[row][k0 + k]
+  __shared__ __align__(16) float Bs[KC][LDB];  // Bs[k][col] = U[i1 + k0 + k][c0 + col]
   const int i2 = i1 + B;
-  const int64_t r0 = (int64_t)blockIdx.x * 64;  // row tiles on x (up to 2^31 - 1)
-  const int c0 = i2 + blockIdx.y * 64;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < B; k0 += KC) {
-    for (int e = threadIdx.x; e < 64 * KC; e += blockDim.x) {
-      const int r = e / KC, k = e % KC;
+  const int64_t r0 = (int64_t)blockIdx.x * TM;
+  const int c0 = i2 + blockIdx.y * TN;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  float4 ra[4], rb[4];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // A slice: 128 rows x 32 k, float4 along k
+      const int e = tid + 256 * q;
+      const int r = e / (KC / 4), k = (e % (KC / 4)) * 4;
       const int64_t gr = r0 + r;
-      Et[k][r] = (gr < m) ? err[gr * B + k0 + k] : 0.0f;
+      ra[q] = (gr < m) ? *reinterpret_cast<const float4*>(err + gr * B + k0 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int e = threadIdx.x; e < 64 * KC; e += blockDim.x) {
-      const int k = e / 64, c = e % 64;
-      Ut[k][c] = (c0 + c < d) ? U[(size_t)(i1 + k0 + k) * d + c0 + c] : 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // B slice: 32 k x 128 columns, float4 along columns
+      const int e = tid + 256 * q;
+      const int k = e / (TN / 4), c = (e % (TN / 4)) * 4;
+      rb[q] = (c0 + c < d) ? *reinterpret_cast<const float4*>(U + (size_t)(i1 + k0 + k) * d + c0 + c)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < KC; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&Et[k][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Ut[k][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int64_t gr = r0 + ty * 4 + p;
-    if (gr >= m) continue;
+  };
+  auto store = [&]() {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int gc = c0 + tx * 4 + q;
-      if (gc < d) w[gr * d + gc] -= acc[p][q];
+      const int e = tid + 256 * q;
+      const int r = e / (KC / 4), k = (e % (KC / 4)) * 4;
+      As[k + 0][r] = ra[q].x;
+      As[k + 1][r] = ra[q].y;
+      As[k + 2][r] = ra[q].z;
+      As[k + 3][r] = ra[q].w;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + 256 * q;
+      const int k = e / (TN / 4), c = (e % (TN / 4)) * 4;
+      *reinterpret_cast<float4*>(&Bs[k][c]) = rb[q];
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[p][q] = 0.0f;
+  fetch(0);
+  for (int k0 = 0; k0 < B; k0 += KC) {
+    __syncthreads();
+    store();
+    __syncthreads();
+    if (k0 + KC < B) fetch(k0 + KC);
+#pragma unroll 4
+    for (int k = 0; k < KC; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[k][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[k][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int64_t gr = r0 + (p < 4 ? ty * 4 + p : 64 + ty * 4 + (p - 4));
+    if (gr >= m) continue;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int gc = c0 + h * 64 + tx * 4;
+      if (gc < d) {
+        float4* dst = reinterpret_cast<float4*>(w + gr * d + gc);
+        float4 o = *dst;
+        o.x -= acc[p][4 * h + 0];
+        o.y -= acc[p][4 * h + 1];
+        o.z -= acc[p][4 * h + 2];
+        o.w -= acc[p][4 * h + 3];
+        *dst = o;
+      }
     }
   }
 }
@@ -407,8 +453,8 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {
-      dim3 grid((unsigned)((m + 63) / 64), (rest + 63) / 64);
-      lazy_update_kernel<B><<<grid, 256, 0, s>>>(ww, m, d, i1, U, err);
+      dim3 grid((unsigned)((m + 127) / 128), (rest + 127) / 128);
+      lazy_gemm_kernel<B><<<grid, 256, 0, s>>>(ww, m, d, i1, U, err);
       GPTQ_LAUNCH_CHECK();
     }
   }
@@ -445,8 +491,10 @@ size_t quantize_workspace(int64_t m, int64_t d, int block_size) {
   return align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * block_size * sizeof(float), 256);
 }
 
-// U of up to 4096^2 fp32 (64 MB) stays in the 126 MB L2, so each CTA can stream it for its own rows.
-bool quantize_fused(int64_t d) { return d <= 4096; }
+// One launch per layer with 8 rows per CTA pays off while rows are few (each CTA streams all of U
+// from L2 for only 8 rows); with many rows the per-block launches run the lazy update as one large
+// GEMM across all rows instead.
+bool quantize_fused(int64_t m, int64_t d) { return d <= 4096 && m <= 2048; }
 
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d64, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
@@ -455,7 +503,7 @@ gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d
   char* ws = static_cast<char*>(workspace);
   float* ww = reinterpret_cast<float*>(ws);
   float* err = reinterpret_cast<float*>(ws + align_up((size_t)m * d * sizeof(float), 256));
-  if (quantize_fused(d)) {
+  if (quantize_fused(m, d)) {
     switch (w_dtype) {
       case GPTQ_FP32: return launch_rows_b<float>(W, m, d, U, cfg, ww, codes, scales, zeros, s);
       case GPTQ_FP16: return launch_rows_b<__half>(W, m, d, U, cfg, ww, codes, scales, zeros, s);

@@ -111,6 +111,7 @@ QUANT_CASES = [
     (64, 512, 4, 256, 128),
     (48, 384, 4, 64, 32),
     (1, 128, 4, 0, 128),
+    (2100, 256, 4, 0, 128),    # many rows: per-block launches with the all-rows lazy GEMM
     (40, 4224, 3, 128, 128),   # wider than 4096: per-block launches instead of the fused kernel
     (24, 4352, 4, 0, 64),
 ]
