@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
               if (r > j) S1[2 * ty + p][4 * tx + q] -= acc2[p][q];
             }
         }
+        __syncthreads();  // the transposition below reads elements other warps just updated
         // S3 <- tile(r, j) transposed, for the triangular solve
         if (r > j) {
           for (int e = tid; e < NB * NB; e += kThreads) S3[e & 31][e >> 5] = S1[e >> 5][e & 31];
@@ -476,10 +477,10 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
   if (!coop) return GPTQ_ERR_CUDA;
   GPTQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prepare_kernel, kThreads, 0));
   if (occ < 1) return GPTQ_ERR_CUDA;
-  // One CTA per SM.  (Two co-resident CTAs per SM gave wrong, run-to-run different results at
-  // d >= 512 although every item of a phase touches disjoint tiles; until that is understood the
-  // launch keeps one CTA per SM, which is exact and bit-reproducible.)
-  const int grid = sms;
+  // Several CTAs per SM hide the L2 latency of the small trailing items of large orders; small
+  // orders have few items per phase and gain nothing but a slower grid barrier from more CTAs.
+  const int per_sm = d64 <= 1024 ? 1 : (occ < 4 ? occ : 4);
+  const int grid = sms * per_sm;
   GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), stream));
   GPTQ_CUDA_TRY(cudaMemsetAsync(ws + 256, 0, 512, stream));  // barrier words and abort flag
   void* args[] = {&a};
