@@ -117,7 +117,7 @@ GPTQ_API size_t gptq_prepare_workspace_size(int64_t d);
  * The GPTQ pages have no counterpart for this call; it exists for callers that cannot allocate
  * device memory themselves, for example a plugin whose host application owns all device memory
  * through its own pool, or a latency-bound path where no allocator may be called.  The scratch the
- * computation needs (about 1 MiB) is a fixed array compiled into this library; every GPU that loads
+ * computation needs (about 4 MiB) is a fixed array compiled into this library; every GPU that loads
  * the library holds it until the process exits.
  *
  *   H, d, damp, U, dev_status, stream: as for gptq_prepare_uinv (U is still caller memory).

@@ -22,9 +22,13 @@ gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, 
                               int32_t accumulate, int32_t* status, void* workspace, cudaStream_t stream);
 
 // A2 + A3
+size_t prepare_blocked_workspace(int64_t d);
+// lookahead: factor the next diagonal block on a library-owned second stream (made once per device)
+gptq_status prepare_blocked_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
+                                   void* workspace, cudaStream_t stream, bool lookahead);
 size_t prepare_workspace(int64_t d);
 gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
-                           void* workspace, cudaStream_t stream);
+                           void* workspace, cudaStream_t stream, bool lookahead = true);
 // same, with the scratch in a static device array (d <= GPTQ_PREPARE_STATIC_MAX_D)
 gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* U, int32_t* status,
                                   cudaStream_t stream);

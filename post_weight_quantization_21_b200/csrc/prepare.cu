@@ -450,13 +450,19 @@ constexpr size_t kSideOffset = 1024;
 
 }  // namespace
 
+// Orders up to kSmallOrder run as the one-launch kernel above (the panel chain dominates); larger
+// orders are dominated by dense block products and take the 128-block path (prepare_blocked.cu).
+constexpr int64_t kSmallOrder = 1024;
+
 size_t prepare_workspace(int64_t d) {
+  if (d > kSmallOrder) return prepare_blocked_workspace(d);
   const int64_t D = (d + NB - 1) / NB;
   return kSideOffset + (size_t)D * NB * NB * sizeof(float);
 }
 
 gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status, void* workspace,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool lookahead) {
+  if (d64 > kSmallOrder) return prepare_blocked_launch(H, d64, damp, U, status, workspace, stream, lookahead);
   const int d = (int)d64;
   char* ws = static_cast<char*>(workspace);
   PrepArgs a;
@@ -477,10 +483,9 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
   if (!coop) return GPTQ_ERR_CUDA;
   GPTQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prepare_kernel, kThreads, 0));
   if (occ < 1) return GPTQ_ERR_CUDA;
-  // Several CTAs per SM hide the L2 latency of the small trailing items of large orders; small
-  // orders have few items per phase and gain nothing but a slower grid barrier from more CTAs.
-  const int per_sm = d64 <= 1024 ? 1 : (occ < 4 ? occ : 4);
-  const int grid = sms * per_sm;
+  // one CTA per SM: the orders served here have few items per phase, and more CTAs only slow the
+  // grid barrier
+  const int grid = sms;
   GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), stream));
   GPTQ_CUDA_TRY(cudaMemsetAsync(ws + 256, 0, 512, stream));  // barrier words and abort flag
   void* args[] = {&a};
@@ -494,13 +499,13 @@ gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, in
 
 namespace gptq {
 // ------------------------------------------------------------------------------------------------
-// Allocation-free variant.  The prepare kernel's scratch (damping value, barrier words, the inverse
-// diagonal blocks: 1 KiB + d/32 * 4 KiB) lives in this file-scope device array instead of a caller
-// workspace, sized for d <= GPTQ_PREPARE_STATIC_MAX_D.  Every GPU that loads the library keeps it for
+// Allocation-free variant.  The prepare step's scratch (damping value, barrier words, the inverse
+// diagonal blocks: at most 1 KiB + d/128 * 64 KiB, about 4 MiB at d = 8192) lives in this file-scope
+// device array instead of a caller workspace, sized for d <= GPTQ_PREPARE_STATIC_MAX_D.  Every GPU that loads the library keeps it for
 // the life of the process.
 namespace {
-constexpr size_t kStaticScratchBytes =
-    kSideOffset + (size_t)(GPTQ_PREPARE_STATIC_MAX_D / NB) * NB * NB * sizeof(float);
+// the 128-block path's need at the largest accepted order (larger than the one-launch kernel's)
+constexpr size_t kStaticScratchBytes = 1024 + (size_t)(GPTQ_PREPARE_STATIC_MAX_D / 128) * 128 * 128 * sizeof(float);
 static __device__ __align__(256) unsigned char g_prepare_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -526,12 +531,13 @@ gptq_status static_scratch(void** out) {
 
 gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* U, int32_t* status,
                                   cudaStream_t stream) {
-  static_assert(kStaticScratchBytes >= kSideOffset + 256 * NB * NB * sizeof(float), "scratch too small");
+  static_assert(kStaticScratchBytes >= kSideOffset + (kSmallOrder / NB) * NB * NB * sizeof(float), "scratch too small");
   void* scratch = nullptr;
   gptq_status st = static_scratch(&scratch);
   if (st != GPTQ_OK) return st;
   if (prepare_workspace(d) > kStaticScratchBytes) return GPTQ_ERR_WORKSPACE;
-  return prepare_launch(H, d, damp, U, status, scratch, stream);
+  // no look-ahead stream here: this variant creates no CUDA objects, so every launch stays on `stream`
+  return prepare_launch(H, d, damp, U, status, scratch, stream, false);
 }
 
 }  // namespace gptq

@@ -1,0 +1,496 @@
+// A2 + A3 for large orders: dampening and U = upper Cholesky factor of Hd^-1 with 128-wide blocks
+// and host-ordered launches (FDE Interviews breakdown of GPTQ, figure "THE IDEA, VISUALLY" step 2,
+// "U = chol(H^-1)"; zhiliyouxian blog, 算法流程 "H = H + lambda * I").
+//
+// Same route as the one-launch kernel (prepare.cu): factor P = J Hd J = L L^T, invert Y = L^-1, and
+// U = J Y J.  Here the work of large orders is dominated by dense block products, so it is spelled
+// as a right-looking blocked Cholesky over 128-column panels followed by a recursive-doubling
+// triangular inverse, each step a launch:
+//   diag_mean, reverse_damp                        lambda, lower(P) = J (H + lambda I) J
+//   factor(0)
+//   for each panel p:
+//     trsm(p)           L(r, p) = P(r, p) L(p,p)^-T for every row block r > p
+//     syrk(p)           P(r, c) -= L(r, p) L(c, p)^T for p < c <= r, except the block (p+1, p+1)
+//     factor(p+1)       one CTA: P(p+1,p+1) - L(p+1,p) L(p+1,p)^T, factored in four 32-wide steps
+//                       (each a one-warp factorisation) and inverted -> side[p+1] = L(p+1,p+1)^-1
+//   leaf_copy           diagonal blocks of P <- side
+//   for g = 1, 2, 4, ...: T = C A^-1, Y21 = -B^-1 T for [[A,0],[C,B]] pairs of g blocks
+//   rotate              U = J Y J
+// factor(p+1) depends only on trsm(p), so it runs on a second stream alongside syrk(p) (look-ahead):
+// the serial chain per panel is trsm + max(syrk, factor) instead of their sum.  The block products
+// run on one 128x128x128 fp32 tile kernel (8x8 outputs per thread).
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gptq {
+namespace {
+
+constexpr int BB = 128;   // block order
+constexpr int LDS = BB + 4;
+constexpr int kSideOff = 1024;
+constexpr int kSub = 32;  // sub-block of the diagonal factorisation
+
+// ------------------------------------------------------------------ lambda and reversed copy
+__global__ void diag_mean_kernel(const float* __restrict__ H, int d, float damp, float* __restrict__ lam) {
+  double s = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) s += (double)H[(size_t)i * d + i];
+  __shared__ double red[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    *lam = (float)((double)damp * t / (double)d);
+  }
+}
+
+__global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const float* __restrict__ lam,
+                                    float* __restrict__ P) {
+  const float l = *lam;
+  for (int i = blockIdx.x; i < d; i += gridDim.x) {
+    const float* src = H + (size_t)(d - 1 - i) * d + (d - 1);
+    float* dst = P + (size_t)i * d;
+    for (int j = threadIdx.x; j <= i; j += blockDim.x) dst[j] = src[-j] + (i == j ? l : 0.0f);
+  }
+}
+
+// ------------------------------------------------------------------ panel factorisation
+// One warp factors a 32x32 block (lower part, stride LDS) and writes its inverse, natural layout,
+// into Li (stride LDS): lane i keeps row i of A, lane c keeps column c of the right-hand sides of
+// L Y = I; right-looking with an unscaled pivot column.
+__device__ void warp_factor_invert_128(const float* A, float* Li, float* colv, float* rsm, int d, int pivot_base,
+                                       int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  float a[kSub], rr[kSub];
+#pragma unroll
+  for (int c = 0; c < kSub; ++c) {
+    a[c] = A[lane * LDS + c];
+    rr[c] = (c == lane) ? 1.0f : 0.0f;
+  }
+#pragma unroll
+  for (int k = 0; k < kSub; ++k) {
+    float* cv = colv + (k & 1) * kSub;
+    cv[lane] = (lane > k) ? a[k] : 0.0f;
+    const float p = __shfl_sync(0xffffffffu, a[k], k);
+    __syncwarp();
+    const float inv = __fdividef(1.0f, p);
+    const float li = a[k] * inv;
+    const float t = rr[k] * inv;
+    if (lane == 0) {
+      rsm[k] = rsqrtf(p);
+      if (!(p > 0.0f && isfinite(p)) && pivot_base + k < d) report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
+    }
+#pragma unroll
+    for (int x4 = (k + 1) & ~3; x4 < kSub; x4 += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(cv + x4);
+      a[x4 + 0] = fmaf(-li, v.x, a[x4 + 0]);
+      a[x4 + 1] = fmaf(-li, v.y, a[x4 + 1]);
+      a[x4 + 2] = fmaf(-li, v.z, a[x4 + 2]);
+      a[x4 + 3] = fmaf(-li, v.w, a[x4 + 3]);
+      rr[x4 + 0] = fmaf(-v.x, t, rr[x4 + 0]);
+      rr[x4 + 1] = fmaf(-v.y, t, rr[x4 + 1]);
+      rr[x4 + 2] = fmaf(-v.z, t, rr[x4 + 2]);
+      rr[x4 + 3] = fmaf(-v.w, t, rr[x4 + 3]);
+    }
+  }
+  __syncwarp();
+  // lane holds column `lane` of the right-hand sides: Linv[i][lane] = rr[i] / sqrt(pivot_i)
+#pragma unroll
+  for (int i = 0; i < kSub; ++i) Li[i * LDS + lane] = (i >= lane) ? rr[i] * rsm[i] : 0.0f;
+  __syncwarp();
+}
+
+// out (M x N, stride LDS) = beta * out + alpha * sum_{k<K} A[m][k] * B(k, n), by all 256 threads;
+// M and N multiples of 32, at most 128.  B(k, n) = B[n][k] (tb) or B[k][n] (!tb).  The output is cut
+// into 32x32 warp tiles; lane (mi, ni) = (lane / 8, lane % 8) of a warp owns rows mi + 4i and
+// columns ni + 8j of its tile, which keeps the shared-memory reads free of bank conflicts with the
+// row stride LDS.  Products are kept in registers and stored after a barrier, so out may alias the
+// inputs.  beta is 0 or 1.
+__device__ void block_mm(float* out, const float* A, const float* B, bool tb, int M, int N, int K, float alpha,
+                         float beta) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mi = lane >> 3, ni = lane & 7;
+  const int wn = N / 32, n_wt = (M / 32) * wn;
+  float r[2][8][4];
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int wt = warp + pass * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) r[pass][i][j] = 0.0f;
+    if (wt < n_wt) {
+      const float* a = A + ((wt / wn) * 32 + mi) * LDS;
+      const int n0 = (wt % wn) * 32 + ni;
+      for (int k = 0; k < K; ++k) {
+        float av[8], bv[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) av[i] = a[4 * i * LDS + k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bv[j] = tb ? B[(n0 + 8 * j) * LDS + k] : B[k * LDS + n0 + 8 * j];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) r[pass][i][j] = fmaf(av[i], bv[j], r[pass][i][j]);
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int wt = warp + pass * 8;
+    if (wt < n_wt) {
+      float* o = out + ((wt / wn) * 32 + mi) * LDS + (wt % wn) * 32 + ni;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float* e = o + 4 * i * LDS + 8 * j;
+          *e = (beta != 0.0f ? *e : 0.0f) + alpha * r[pass][i][j];
+        }
+    }
+  }
+  __syncthreads();
+}
+
+// Factors the 128x128 diagonal block p and writes side[p] = L(p,p)^-1 (row-major, zeros above the
+// diagonal).  When p > 0 the block first receives its last update, P(p,p) - L(p,p-1) L(p,p-1)^T (the
+// trailing update of panel p-1 leaves this block out, so its factorisation can run alongside).
+// Runs as block 0 of the panel-(p-1) update launch; 256 threads, dynamic shared memory.
+__device__ void factor_block(const float* P, int d, int p, float* side, int32_t* status, float* sm) {
+  float* A = sm;                  // [128][LDS]
+  float* Li = sm + BB * LDS;      // [128][LDS]
+  float* S = Li + BB * LDS;       // [128][LDS]: L(p, p-1), then scratch
+  float* colv = S + BB * LDS;     // 2 x 32
+  float* rsm = colv + 2 * kSub;   // 32
+  const int p0 = p * BB;
+  // batched loads: every thread issues its 16 loads before storing
+  for (int base = 0; base < BB * BB; base += 16 * 256) {
+    float va[16], vs[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = base + threadIdx.x + q * 256;
+      const int i = e / BB, c = e % BB;
+      const int gi = p0 + i, gc = p0 + c;
+      va[q] = (gi < d && gc < d) ? ((c <= i) ? P[(size_t)gi * d + gc] : 0.0f) : ((i == c) ? 1.0f : 0.0f);
+      vs[q] = (p > 0 && gi < d && gc - BB < d) ? P[(size_t)gi * d + gc - BB] : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = base + threadIdx.x + q * 256;
+      A[(e / BB) * LDS + e % BB] = va[q];
+      S[(e / BB) * LDS + e % BB] = vs[q];
+      Li[(e / BB) * LDS + e % BB] = 0.0f;
+    }
+  }
+  __syncthreads();
+  if (p > 0) block_mm(A, S, S, true, BB, BB, BB, -1.0f, 1.0f);  // A -= L(p,p-1) L(p,p-1)^T
+  for (int s = 0; s < BB / kSub; ++s) {
+    float* Ass = A + s * kSub * LDS + s * kSub;
+    if (threadIdx.x < 32) warp_factor_invert_128(Ass, Li + s * kSub * LDS + s * kSub, colv, rsm, d, p0 + s * kSub, status);
+    __syncthreads();
+    const int rest = BB - (s + 1) * kSub;
+    if (rest > 0) {
+      float* Ats = A + (s + 1) * kSub * LDS + s * kSub;
+      block_mm(Ats, Ats, Li + s * kSub * LDS + s * kSub, true, rest, kSub, kSub, 1.0f, 0.0f);  // L(t, s)
+      float* Atr = A + (s + 1) * kSub * LDS + (s + 1) * kSub;
+      block_mm(Atr, Ats, Ats, true, rest, rest, kSub, -1.0f, 1.0f);  // trailing part of the block
+    }
+  }
+  // [[A,0],[C,B]]^-1 = [[A^-1, 0], [-B^-1 C A^-1, B^-1]], 32 -> 64 -> 128
+  for (int h = kSub; h < BB; h *= 2) {
+    for (int a0 = 0; a0 < BB; a0 += 2 * h) {
+      const int b0 = a0 + h;
+      block_mm(S, A + b0 * LDS + a0, Li + a0 * LDS + a0, false, h, h, h, 1.0f, 0.0f);
+      block_mm(Li + b0 * LDS + a0, Li + b0 * LDS + b0, S, false, h, h, h, -1.0f, 0.0f);
+    }
+  }
+  float* out = side + (size_t)p * BB * BB;
+  for (int e = threadIdx.x; e < BB * BB; e += blockDim.x) {
+    const int i = e / BB, c = e % BB;
+    out[e] = (c <= i) ? Li[i * LDS + c] : 0.0f;
+  }
+}
+
+constexpr int kFactorSmem = (3 * BB * LDS + 3 * kSub) * sizeof(float);
+
+__global__ void __launch_bounds__(256) factor_kernel(const float* __restrict__ P, int d, int p, float* __restrict__ side,
+                                                     int32_t* status) {
+  extern __shared__ __align__(16) float fsm[];
+  factor_block(P, d, p, side, status, fsm);
+}
+
+// ------------------------------------------------------------------ 128x128x128 tile products
+enum TileMode { kTrsm = 0, kSyrk = 1, kTrtriT = 2, kTrtriY = 3 };
+
+struct TileArgs {
+  float* P;
+  const float* side;
+  int d, D;   // order, 128-blocks
+  int p;      // panel (trsm, syrk)
+  int g;      // half size in blocks (trtri levels)
+  int skip;   // syrk: leading output tiles left out (the next diagonal block, factored alongside)
+};
+
+__device__ __forceinline__ float ld_or0(const float* base, int64_t r, int64_t c, int d) {
+  return (r < d && c < d) ? base[r * d + c] : 0.0f;
+}
+
+// Output tile C (128x128 at block (ri, ci)) = sum over K blocks of A(ri, k) B(k, ci):
+//   trsm:    A = P(r, p),  B(k, n) = side[p][n][k]            -> P(r, p) = acc
+//   syrk:    A = P(r, p),  B(k, n) = P(c, p)[n][k]            -> P(r, c) -= acc
+//   trtriT:  A = P(r, k),  B = P(k, c) (k from c to a1-1)     -> P(c, r) = acc^T   (T parked transposed)
+//   trtriY:  A = P(r, k),  B(k, n) = P(c, k)[n][k] (k <= r)   -> P(r, c) = -acc
+template <int MODE>
+__global__ void __launch_bounds__(256) tile_gemm_kernel(const TileArgs a) {
+  constexpr int KC = 32;
+  __shared__ __align__(16) float As[KC][BB + 4];  // As[k][m]
+  __shared__ __align__(16) float Bs[KC][BB + 4];  // Bs[k][n]
+  const int d = a.d;
+  int ri = 0, ci = 0, kb0 = 0, kb1 = 1;
+  const int bid = blockIdx.x + (MODE == kSyrk ? a.skip : 0);
+  if (MODE == kTrsm) {
+    ri = a.p + 1 + bid;
+    ci = a.p;
+  } else if (MODE == kSyrk) {
+    int rr = (int)((sqrt(8.0 * (double)bid + 1.0) - 1.0) * 0.5);
+    while ((rr + 1) * (rr + 2) / 2 <= bid) ++rr;
+    while (rr * (rr + 1) / 2 > bid) --rr;
+    ri = a.p + 1 + rr;
+    ci = a.p + 1 + (bid - rr * (rr + 1) / 2);
+  } else {
+    const int per_pair = a.g * a.g;
+    const int q = bid / per_pair, t = bid % per_pair;
+    const int a0 = q * 2 * a.g, b0 = a0 + a.g, b1 = min(a0 + 2 * a.g, a.D);
+    ri = b0 + t / a.g;
+    ci = a0 + t % a.g;
+    if (ri >= b1) return;
+    if (MODE == kTrtriT) {
+      kb0 = ci;
+      kb1 = b0;  // A^-1 (k, c) is zero for k < c
+    } else {
+      kb0 = b0;
+      kb1 = ri + 1;  // B^-1 (r, k) is zero for k > r
+    }
+  }
+  const int64_t r0 = (int64_t)ri * BB, c0 = (int64_t)ci * BB;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  float ra[16], rb[16];
+  // slice s of the K range: block kb = kb0 + s / 4, columns (s % 4) * 32 .. +32 of that block
+  auto fetch = [&](int s) {
+    const int kb = kb0 + s / (BB / KC);
+    const int64_t k0 = (int64_t)kb * BB + (s % (BB / KC)) * KC;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {  // A: 128 rows (m) x 32 k, read along k
+      const int e = tid + 256 * q;
+      const int m = e / KC, k = e % KC;
+      const int64_t acol = (MODE == kTrsm || MODE == kSyrk) ? (int64_t)a.p * BB + (k0 - (int64_t)kb * BB) + k : k0 + k;
+      ra[q] = ld_or0(a.P, r0 + m, acol, d);
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = tid + 256 * q;
+      if (MODE == kTrtriT) {  // B natural: rows k, columns n
+        const int k = e / BB, n = e % BB;
+        rb[q] = ld_or0(a.P, k0 + k, c0 + n, d);
+      } else {                // B stored [n][k]
+        const int n = e / KC, k = e % KC;
+        if (MODE == kTrsm) {
+          const int64_t kk = k0 - (int64_t)kb * BB + k;
+          rb[q] = a.side[((size_t)a.p * BB + n) * BB + kk];
+        } else if (MODE == kSyrk) {
+          rb[q] = ld_or0(a.P, c0 + n, (int64_t)a.p * BB + (k0 - (int64_t)kb * BB) + k, d);
+        } else {  // trtriY: T(k, c) stored at P(c, k)
+          rb[q] = ld_or0(a.P, c0 + n, k0 + k, d);
+        }
+      }
+    }
+  };
+  auto store = [&]() {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = tid + 256 * q;
+      As[e % KC][e / KC] = ra[q];
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = tid + 256 * q;
+      if (MODE == kTrtriT)
+        Bs[e / BB][e % BB] = rb[q];
+      else
+        Bs[e % KC][e / KC] = rb[q];
+    }
+  };
+  const int n_slices = (kb1 - kb0) * (BB / KC);
+  fetch(0);
+  for (int s = 0; s < n_slices; ++s) {
+    __syncthreads();
+    store();
+    __syncthreads();
+    if (s + 1 < n_slices) fetch(s + 1);
+#pragma unroll 4
+    for (int k = 0; k < KC; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[k][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[k][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t gr = r0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t gc = c0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
+      if (gr >= d || gc >= d) continue;
+      if (MODE == kTrsm) {
+        a.P[gr * d + gc] = acc[i][j];
+      } else if (MODE == kSyrk) {
+        a.P[gr * d + gc] -= acc[i][j];
+      } else if (MODE == kTrtriT) {
+        a.P[gc * d + gr] = acc[i][j];
+      } else {
+        a.P[gr * d + gc] = -acc[i][j];
+      }
+    }
+  }
+}
+
+// diagonal 128-blocks of P <- their inverses (zeros above the diagonal)
+__global__ void leaf_copy_kernel(float* __restrict__ P, int d, const float* __restrict__ side) {
+  const int p = blockIdx.x;
+  const float* src = side + (size_t)p * BB * BB;
+  for (int e = threadIdx.x; e < BB * BB; e += blockDim.x) {
+    const int i = e / BB, c = e % BB;
+    const int64_t gi = (int64_t)p * BB + i, gc = (int64_t)p * BB + c;
+    if (gi < d && gc < d) P[gi * d + gc] = src[e];
+  }
+}
+
+// U = J Y J in place: lower block triangle -> upper, strict lower part zeroed, diagonal reversed
+__global__ void rotate_kernel(float* __restrict__ P, int d) {
+  for (int i = blockIdx.x; i < d; i += gridDim.x) {
+    float* row = P + (size_t)i * d;
+    float* mirror = P + (size_t)(d - 1 - i) * d + (d - 1);
+    for (int j = threadIdx.x; j <= i; j += blockDim.x) {
+      if (j < i) {
+        mirror[-j] = row[j];
+        row[j] = 0.0f;
+      } else if (i < d - 1 - i) {
+        const float va = row[i], vb = mirror[-i];
+        row[i] = vb;
+        mirror[-i] = va;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t prepare_blocked_workspace(int64_t d) {
+  const int64_t D = (d + BB - 1) / BB;
+  return kSideOff + (size_t)D * BB * BB * sizeof(float);
+}
+
+namespace {
+
+// The look-ahead stream and its two events, one set per device, made on first use.
+struct LookAhead {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+std::mutex g_lookahead_mu;
+LookAhead g_lookahead[64];
+
+}  // namespace
+
+gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status, void* workspace,
+                                   cudaStream_t s, bool lookahead) {
+  const int d = (int)d64;
+  const int D = (d + BB - 1) / BB;
+  char* ws = static_cast<char*>(workspace);
+  float* lam = reinterpret_cast<float*>(ws);
+  float* side = reinterpret_cast<float*>(ws + kSideOff);
+  int dev = 0, sms = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFactorSmem));
+  std::unique_lock<std::mutex> hold(g_lookahead_mu, std::defer_lock);
+  LookAhead* la = nullptr;
+  if (lookahead && dev < 64) {
+    hold.lock();  // the events are shared: one enqueue sequence at a time
+    la = &g_lookahead[dev];
+    if (la->side == nullptr) {
+      GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&la->side, cudaStreamNonBlocking));
+      GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&la->fork, cudaEventDisableTiming));
+      GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&la->join, cudaEventDisableTiming));
+    }
+  }
+  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), s));
+  diag_mean_kernel<<<1, 1024, 0, s>>>(H, d, damp, lam);
+  GPTQ_LAUNCH_CHECK();
+  reverse_damp_kernel<<<sms * 4, 256, 0, s>>>(H, d, lam, U);
+  GPTQ_LAUNCH_CHECK();
+  factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, 0, side, status);
+  GPTQ_LAUNCH_CHECK();
+  TileArgs ta{U, side, d, D, 0, 0, 1};
+  for (int p = 0; p + 1 < D; ++p) {
+    const int below = D - p - 1;
+    ta.p = p;
+    tile_gemm_kernel<kTrsm><<<below, 256, 0, s>>>(ta);
+    GPTQ_LAUNCH_CHECK();
+    cudaStream_t fs = s;
+    if (la != nullptr) {
+      GPTQ_CUDA_TRY(cudaEventRecord(la->fork, s));
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
+      fs = la->side;
+      factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, side, status);
+      GPTQ_LAUNCH_CHECK();
+      GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
+    }
+    const int tiles = below * (below + 1) / 2 - 1;
+    if (tiles > 0) {
+      tile_gemm_kernel<kSyrk><<<tiles, 256, 0, s>>>(ta);
+      GPTQ_LAUNCH_CHECK();
+    }
+    if (la != nullptr) {
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+    } else {
+      factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, side, status);
+      GPTQ_LAUNCH_CHECK();
+    }
+  }
+  leaf_copy_kernel<<<D, 256, 0, s>>>(U, d, side);
+  GPTQ_LAUNCH_CHECK();
+  for (int g = 1; g < D; g *= 2) {
+    const int pairs = (D + 2 * g - 1) / (2 * g);
+    ta.g = g;
+    tile_gemm_kernel<kTrtriT><<<pairs * g * g, 256, 0, s>>>(ta);
+    GPTQ_LAUNCH_CHECK();
+    tile_gemm_kernel<kTrtriY><<<pairs * g * g, 256, 0, s>>>(ta);
+    GPTQ_LAUNCH_CHECK();
+  }
+  rotate_kernel<<<sms * 4, 256, 0, s>>>(U, d);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

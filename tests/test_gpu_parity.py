@@ -74,7 +74,7 @@ def test_hessian_full_size_opt125m_layer():
 
 
 # ------------------------------------------------------------------------------------------ A2 + A3
-@pytest.mark.parametrize("d", [1, 5, 31, 33, 64, 128, 200, 768, 1000, 2048, 4224])
+@pytest.mark.parametrize("d", [1, 5, 31, 33, 64, 128, 200, 768, 1000, 1100, 1500, 2048, 4224])
 def test_prepare_matches_oracle(d):
     n = max(4 * d, 64)
     X = _x(n, d, torch.float64, seed=d)
