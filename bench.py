@@ -203,10 +203,9 @@ def main():
 
     solver = g.LayerSolver(L.m, L.d, L.n_tokens, L.bits, L.group_size, L.block_size, L.damp, L.x_dtype,
                            L.w_dtype, device=dev)
-    W = wl.make_w(L)
-    X = wl.make_x(L)
-    solver.W.copy_(W)
-    solver.X.copy_(X)
+    # seeded inputs made on the device (the large layers' X is tens of GB); host copies below
+    solver.W.copy_(wl.make_w(L, device=dev))
+    wl.make_x(L, device=dev, out=solver.X)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -259,8 +258,10 @@ def main():
     value = world * L.m * L.d / (ms_per_step * 1e-3)
 
     # end to end through the host: pinned inputs in, packed codes + grids out, every step
-    W_h = W.pin_memory()
-    X_h = X.pin_memory()
+    W_h = torch.empty(solver.W.shape, dtype=solver.W.dtype).pin_memory()
+    X_h = torch.empty(solver.X.shape, dtype=solver.X.dtype).pin_memory()
+    W_h.copy_(solver.W)
+    X_h.copy_(solver.X)
     n_groups = 1 if L.group_size == 0 else L.d // L.group_size
     out_p = torch.empty(L.m, L.d * L.bits // 32, dtype=torch.int32).pin_memory()
     out_s = torch.empty(L.m, n_groups, dtype=torch.float32).pin_memory()
@@ -320,7 +321,8 @@ def main():
             "phase_roofline_ms": roof_ms, "end_to_end_roofline_frac": roof_ms / ms_per_step,
             "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        W64 = W.double().numpy()
+        W64 = W_h.double().numpy()
+        X = X_h
         cores, blas = cores_info()
         t0 = time.perf_counter()
         n = 0

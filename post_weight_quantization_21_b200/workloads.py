@@ -143,6 +143,29 @@ def make_x_chunk(layer: Layer, c: int, device="cpu") -> torch.Tensor:
     return x.to(layer.x_dtype)
 
 
+def make_upper(d: int, seed: int, device="cpu", rows_per_chunk: int = 1024) -> torch.Tensor:
+    """A seeded upper-triangular fp32 matrix [d, d] with a positive diagonal, used as a stand-in U input.
+
+    Diagonal ~ U(0.5, 1.5); entry (i, j > i) = U_ii * 0.5 * N(0, 1) / (1 + j - i), so each row's
+    off-diagonal weights decay away from the diagonal the way a correlated layer's do.  Rows are drawn
+    in chunks of ``rows_per_chunk``, chunk c from seed * 1000003 + c, on ``device``.
+    """
+    U = torch.empty(d, d, dtype=torch.float32, device=device)
+    col = torch.arange(d, device=device, dtype=torch.float32)
+    for c, r0 in enumerate(range(0, d, rows_per_chunk)):
+        r1 = min(d, r0 + rows_per_chunk)
+        g = _gen(seed * 1000003 + c, device)
+        diag = torch.rand(r1 - r0, generator=g, device=device, dtype=torch.float32) + 0.5
+        off = torch.randn(r1 - r0, d, generator=g, device=device, dtype=torch.float32)
+        rows = torch.arange(r0, r1, device=device, dtype=torch.float32)[:, None]
+        dist = col[None, :] - rows
+        blk = diag[:, None] * 0.5 * off / (1.0 + dist.clamp_min(0.0))
+        blk = torch.where(dist > 0, blk, torch.zeros((), device=device))
+        blk[torch.arange(r1 - r0, device=device), torch.arange(r0, r1, device=device)] = diag
+        U[r0:r1] = blk
+    return U
+
+
 def make_x(layer: Layer, device="cpu", out: torch.Tensor | None = None) -> torch.Tensor:
     """The whole X [n_tokens, d]; written into ``out`` when given (e.g. a preallocated device buffer)."""
     if out is None:

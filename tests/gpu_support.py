@@ -41,7 +41,8 @@ def prepare(H: torch.Tensor, damp: float = 0.01, expect_ok: bool = True):
     return U, code, detail
 
 
-def quantize(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int, block_size: int):
+def quantize(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int, block_size: int, rows=None):
+    """Codes, scales, zeros of the whole layer (of ``rows`` only when given) as int64/fp32 host arrays."""
     m, d = W.shape
     n_groups = 1 if group_size == 0 else d // group_size
     codes = torch.empty(m, d, dtype=torch.uint8, device=W.device)
@@ -51,6 +52,9 @@ def quantize(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int, block
                      device=W.device)
     g.gptq_quantize_layer(W, U, codes, scales, zeros, ws, bits, group_size, block_size)
     torch.cuda.synchronize()
+    if rows is not None:
+        idx = torch.as_tensor(rows, device=W.device)
+        codes, scales, zeros = codes[idx], scales[idx], zeros[idx]
     return codes.cpu().numpy().astype(np.int64), scales.cpu().numpy(), zeros.cpu().numpy().astype(np.int64)
 
 

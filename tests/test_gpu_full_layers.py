@@ -4,12 +4,14 @@ The oracle cannot afford an fp64 H of every large layer end to end, so each stag
 what it can compute exactly, and no stage takes an input from the CUDA path:
 
 * H: the full GPU Hessian against fp64 on sampled 128x128 blocks (diagonal, off-diagonal and
-  outlier-channel blocks), all 262,144 tokens.
+  outlier-channel blocks), all 262,144 tokens; only the sampled channels leave the device.
 * U: the trailing k x k principal block of U depends only on the trailing k x k block of the
   dampened Hessian (write Hd = R R^T with R upper: U = R^-1 and U_22 = R_22^-1).  The oracle builds
   that block (and the damping from all column norms) from X in fp64 and factors it.
 * Column loop: the full m x d layer quantized on the GPU with an oracle U (from a token subsample
-  of the same inputs) against the oracle's quantization of the same rows with the same U.
+  of the same inputs) against the oracle's quantization of the same rows with the same U.  At
+  d = 49152 the oracle cannot factor a Hessian, so the column loop there takes a seeded dense
+  upper-triangular U (an input of the quantize call like any other) on both sides.
 * End to end on the 4096-wide layer: all stages chained on the GPU against the fp64 oracle.
 """
 import numpy as np
@@ -24,6 +26,7 @@ import gpu_support as S
 pytestmark = pytest.mark.gpu
 
 LARGE = ["llama7b_q_4096x4096", "llama7b_up_11008x4096", "llama7b_down_4096x11008"]
+WIDEST = "opt175b_fc2_12288x49152"
 
 
 def _blocks(d, oc, rng):
@@ -33,25 +36,34 @@ def _blocks(d, oc, rng):
     return [(min(a, b), max(a, b)) for a, b in pairs]
 
 
-def _x_cpu_chunks(X, step=16384):
+def _x_cpu_chunks(X, step=16384, cols=None):
+    idx = None if cols is None else torch.as_tensor(cols, device=X.device)
     for t0 in range(0, X.shape[0], step):
-        yield X[t0:t0 + step].cpu().double().numpy()
+        Xc = X[t0:t0 + step]
+        if idx is not None:
+            Xc = Xc.index_select(1, idx)
+        yield Xc.cpu().double().numpy()
 
 
-@pytest.mark.parametrize("name", ["llama7b_q_4096x4096", "llama7b_down_4096x11008"])
+@pytest.mark.parametrize("name", ["llama7b_q_4096x4096", "llama7b_down_4096x11008", WIDEST])
 def test_hessian_sampled_blocks(name):
     L = wl.LAYERS[name]
     X = wl.make_x(L, device="cuda")
     H = S.hessian(X)
     rng = np.random.default_rng(0)
     blocks = _blocks(L.d, wl.outlier_channels(L).numpy(), rng)
+    got = {(a, b): H[a:a + 128, b:b + 128].double().cpu().numpy() for a, b in blocks}
+    del H
+    starts = sorted({s for pair in blocks for s in pair})
+    pos = {s0: 128 * k for k, s0 in enumerate(starts)}
+    cols = np.concatenate([np.arange(s0, s0 + 128) for s0 in starts])
     ref = {p: np.zeros((128, 128)) for p in blocks}
-    for Xc in _x_cpu_chunks(X):
+    for Xc in _x_cpu_chunks(X, cols=cols):
         for (a, b) in blocks:
-            ref[(a, b)] += 2.0 * Xc[:, a:a + 128].T @ Xc[:, b:b + 128]
+            ref[(a, b)] += 2.0 * Xc[:, pos[a]:pos[a] + 128].T @ Xc[:, pos[b]:pos[b] + 128]
     num = den = 0.0
     for (a, b), R in ref.items():
-        G = H[a:a + 128, b:b + 128].double().cpu().numpy()
+        G = got[(a, b)]
         if a == b:
             iu = np.triu_indices(128)
             G, R = G[iu], R[iu]
@@ -60,16 +72,18 @@ def test_hessian_sampled_blocks(name):
     assert np.sqrt(num / den) <= S.H_REL_FRO
 
 
-@pytest.mark.parametrize("name", ["llama7b_q_4096x4096", "llama7b_down_4096x11008"])
-def test_prepare_trailing_block(name):
+@pytest.mark.parametrize("name,k", [("llama7b_q_4096x4096", 512), ("llama7b_down_4096x11008", 512),
+                                    (WIDEST, 2048)])
+def test_prepare_trailing_block(name, k):
     L = wl.LAYERS[name]
-    k = 512
     X = wl.make_x(L, device="cuda")
     H = S.hessian(X)
     U = S.prepare(H, L.damp)[-k:, -k:].double().cpu().numpy()
+    del H
+    torch.cuda.empty_cache()
     colsq = np.zeros(L.d)
     Hk = np.zeros((k, k))
-    for Xc in _x_cpu_chunks(X):
+    for Xc in _x_cpu_chunks(X, step=16384 if L.d <= 16384 else 2048):
         colsq += np.einsum("ij,ij->j", Xc, Xc)
         Hk += 2.0 * Xc[:, -k:].T @ Xc[:, -k:]
     lam = L.damp * np.mean(2.0 * colsq)
@@ -98,6 +112,21 @@ def test_quantize_full_layer_with_oracle_u(name):
     st = S.compare_quantization((gpu[0][rows], gpu[1][rows], gpu[2][rows]), ref, L.group_size, Wr, Hs,
                                 label=name)
     print(name, st)
+
+
+def test_quantize_widest_layer_with_seeded_u():
+    L = wl.LAYERS[WIDEST]
+    rows = np.sort(np.random.default_rng(3).choice(L.m, size=256, replace=False))
+    U = wl.make_upper(L.d, seed=11, device="cuda")
+    W = wl.make_w(L, device="cuda")
+    gpu = S.quantize(W, U, L.bits, L.group_size, L.block_size, rows=rows)
+    Wr = W[torch.as_tensor(rows, device=W.device)].double().cpu().numpy()
+    del W
+    U64 = U.cpu().double().numpy()
+    del U
+    ref = oracle.gptq_quantize(Wr, U64, L.bits, L.group_size, L.block_size)
+    st = S.compare_quantization(gpu, ref, L.group_size, label=WIDEST)
+    print(WIDEST, st)
 
 
 def test_end_to_end_llama_q_layer():
