@@ -343,7 +343,8 @@ def main():
 
 
 def hessian_sources():
-    return ["post_weight_quantization_21_b200/csrc/hessian.cu", "post_weight_quantization_21_b200/csrc/hessian_tc.cu"]
+    return ["post_weight_quantization_21_b200/csrc/hessian.cu", "post_weight_quantization_21_b200/csrc/hessian_tc.cu",
+            "post_weight_quantization_21_b200/csrc/tc_common.cuh"]
 
 
 if __name__ == "__main__":

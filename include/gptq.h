@@ -37,7 +37,7 @@
 extern "C" {
 #endif
 
-#define GPTQ_ABI_VERSION 1
+#define GPTQ_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define GPTQ_API __attribute__((visibility("default")))
@@ -59,6 +59,8 @@ typedef enum { GPTQ_BF16 = 0, GPTQ_FP16 = 1, GPTQ_FP32 = 2 } gptq_dtype;
 
 /* Flags of gptq_quant_cfg.flags. */
 #define GPTQ_FLAG_ACT_ORDER 1u /* reorder columns by descending diag(H) ("desc_act"); unsupported */
+#define GPTQ_FLAG_FP32_FMA 2u  /* lazy block updates on the fp32 FMA units instead of the tensor cores
+                                  (3xTF32: tf32 hi/lo splits of both operands, fp32 accumulation) */
 
 /* Quantization settings of one layer (zhiliyouxian blog, 实践指南: bits, group_size, desc_act;
  * agent.csdn.net "GPTQ量化参数搜索工具", 关键参数说明 table: bits, group_size, zero point;
@@ -147,13 +149,18 @@ GPTQ_API gptq_status gptq_prepare_uinv_static(const float* H, int64_t d, float d
  *   codes      [m, d] uint8 output, one code per weight.
  *   scales     [m, n_groups] fp32 output, n_groups = group_size ? d / group_size : 1.
  *   zeros      [m, n_groups] int32 output.
+ *   dev_status device int32[2]: cleared at the start of the call; a kernel that gives up a bounded
+ *              wait records GPTQ_ERR_TIMEOUT there (read with gptq_read_status).
  *   workspace  >= gptq_quantize_workspace_size(m, d, cfg) bytes, 256-byte aligned (holds the
  *              working copy of W in fp32 and the per-block errors).
  *   Requires d % 32 == 0 and d % block_size == 0.  flags & GPTQ_FLAG_ACT_ORDER -> UNSUPPORTED.
+ *   The lazy block updates run on the tensor cores as 3xTF32 products (each operand split into a
+ *   tf32 high part and a tf32 remainder, three MMAs per product, fp32 accumulation: about the
+ *   accuracy of fp32 FMA); flags & GPTQ_FLAG_FP32_FMA selects fp32 FMA units instead.
  * ------------------------------------------------------------------------------------------ */
 GPTQ_API gptq_status gptq_quantize_layer(const void* W, int32_t w_dtype, int64_t m, int64_t d,
                                 const float* U, const gptq_quant_cfg* cfg, uint8_t* codes,
-                                float* scales, int32_t* zeros, void* workspace,
+                                float* scales, int32_t* zeros, int32_t* dev_status, void* workspace,
                                 size_t workspace_bytes, void* stream);
 GPTQ_API size_t gptq_quantize_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* cfg);
 

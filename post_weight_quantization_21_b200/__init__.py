@@ -31,6 +31,7 @@ GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_UNSUPPORTED, GPTQ_ERR_NOT_PD = 0, 1, 2, 3
 GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
 GPTQ_BF16, GPTQ_FP16, GPTQ_FP32 = 0, 1, 2
 GPTQ_FLAG_ACT_ORDER = 1
+GPTQ_FLAG_FP32_FMA = 2
 
 _DTYPES = {torch.bfloat16: GPTQ_BF16, torch.float16: GPTQ_FP16, torch.float32: GPTQ_FP32}
 
@@ -48,7 +49,7 @@ ABI_FUNCTIONS = {
     "gptq_prepare_workspace_size": (_sz, [_i64]),
     "gptq_prepare_uinv_static": (_i32, [_vp, _i64, _f32, _vp, _vp, _vp]),
     "gptq_quantize_layer": (_i32, [_vp, _i32, _i64, _i64, _vp, ctypes.POINTER(QuantCfg), _vp, _vp, _vp,
-                                   _vp, _sz, _vp]),
+                                   _vp, _vp, _sz, _vp]),
     "gptq_quantize_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
     "gptq_pack": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp]),
     "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
@@ -161,15 +162,15 @@ def gptq_quantize_workspace_size(m: int, d: int, bits: int, group_size: int, blo
 
 
 def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
-                        zeros: torch.Tensor, workspace: torch.Tensor, bits: int, group_size: int = 0,
-                        block_size: int = 128, flags: int = 0, stream=None):
+                        zeros: torch.Tensor, status: torch.Tensor, workspace: torch.Tensor, bits: int,
+                        group_size: int = 0, block_size: int = 128, flags: int = 0, stream=None):
     """Column loop with lazy block updates: fills codes [m, d] u8, scales/zeros [m, n_groups]."""
-    for t, n in ((W, "W"), (U, "U"), (codes, "codes"), (scales, "scales"), (zeros, "zeros")):
+    for t, n in ((W, "W"), (U, "U"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"), (status, "status")):
         _contig(t, n)
     m, d = W.shape
     c = _cfg(bits, group_size, block_size, flags)
     st = lib().gptq_quantize_layer(_ptr(W), _DTYPES[W.dtype], m, d, _ptr(U), ctypes.byref(c), _ptr(codes),
-                                   _ptr(scales), _ptr(zeros), _ptr(workspace),
+                                   _ptr(scales), _ptr(zeros), _ptr(status), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "gptq_quantize_layer")
 
@@ -201,8 +202,8 @@ class LayerSolver:
     """
 
     def __init__(self, m: int, d: int, n_tokens: int, bits: int, group_size: int = 0, block_size: int = 128,
-                 damp: float = 0.01, x_dtype=torch.bfloat16, w_dtype=torch.float16, device="cuda"):
-        self.m, self.d, self.n_tokens = m, d, n_tokens
+                 damp: float = 0.01, x_dtype=torch.bfloat16, w_dtype=torch.float16, device="cuda", flags: int = 0):
+        self.m, self.d, self.n_tokens, self.flags = m, d, n_tokens, flags
         self.bits, self.group_size, self.block_size, self.damp = bits, group_size, block_size, damp
         n_groups = 1 if group_size == 0 else d // group_size
         dev = torch.device(device)
@@ -227,8 +228,8 @@ class LayerSolver:
         gptq_prepare_uinv(self.H, self.U, self.status, self.workspace, self.damp, stream)
 
     def quantize(self, stream=None):
-        gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.workspace, self.bits,
-                            self.group_size, self.block_size, 0, stream)
+        gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.status, self.workspace,
+                            self.bits, self.group_size, self.block_size, self.flags, stream)
 
     def pack(self, stream=None):
         gptq_pack(self.codes, self.bits, self.packed, stream)

@@ -25,7 +25,7 @@ gptq_status check_cfg(const gptq_quant_cfg* cfg, int64_t d) {
   if (cfg->bits < 2 || cfg->bits > 4) return GPTQ_ERR_ARG;
   if (cfg->block_size != 32 && cfg->block_size != 64 && cfg->block_size != 128) return GPTQ_ERR_ARG;
   if (cfg->flags & GPTQ_FLAG_ACT_ORDER) return GPTQ_ERR_UNSUPPORTED;
-  if (cfg->flags & ~GPTQ_FLAG_ACT_ORDER) return GPTQ_ERR_ARG;
+  if (cfg->flags & ~(GPTQ_FLAG_ACT_ORDER | GPTQ_FLAG_FP32_FMA)) return GPTQ_ERR_ARG;
   if (d % cfg->block_size) return GPTQ_ERR_ARG;
   const int g = cfg->group_size;
   if (g < 0) return GPTQ_ERR_ARG;
@@ -112,17 +112,18 @@ size_t gptq_quantize_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* 
 
 gptq_status gptq_quantize_layer(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U,
                                 const gptq_quant_cfg* cfg, uint8_t* codes, float* scales, int32_t* zeros,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+                                int32_t* dev_status, void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dtype(w_dtype) || m <= 0 || d <= 0 || d > kMaxDim || m > kMaxDim * 64 || d % 32)
     return GPTQ_ERR_ARG;
   gptq_status st = check_cfg(cfg, d);
   if (st != GPTQ_OK) return st;
-  if (!W || !U || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
-  if (!aligned(W, dtype_size(w_dtype)) || !aligned(U, 16) || !aligned(scales, 4) || !aligned(zeros, 4))
+  if (!W || !U || !codes || !scales || !zeros || !dev_status) return GPTQ_ERR_ARG;
+  if (!aligned(W, dtype_size(w_dtype)) || !aligned(U, 16) || !aligned(scales, 4) || !aligned(zeros, 4) ||
+      !aligned(dev_status, 4))
     return GPTQ_ERR_ARG;
   const size_t need = gptq::quantize_workspace(m, d, cfg->block_size);
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return GPTQ_ERR_WORKSPACE;
-  return gptq::quantize_launch(W, w_dtype, m, d, U, *cfg, codes, scales, zeros, workspace,
+  return gptq::quantize_launch(W, w_dtype, m, d, U, *cfg, codes, scales, zeros, dev_status, workspace,
                                static_cast<cudaStream_t>(stream));
 }
 

@@ -17,11 +17,8 @@
 //               partial) to global memory.
 // Every mbarrier wait is bounded: on a timeout the kernel records GPTQ_ERR_TIMEOUT, lets the
 // other roles leave, waits (bounded) for its own TMA copies and MMAs in flight, frees TMEM, returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace gptq {
 namespace {
@@ -40,7 +37,6 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int kPlanSMs = 148;
 constexpr int kMinTokensPerSplit = 4096;
 constexpr int kChunkTokens = 1024;  // flush period of the TMEM accumulator
-constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 2 GHz
 
 struct TcPlan {
   int nbi, nbj, tiles, splits, units;
@@ -91,83 +87,7 @@ struct TcArgs {
   int32_t* status;
 };
 
-// ------------------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for the phase with the given parity.  Gives up (returns false) when another role has
-// aborted, or after kWaitCycles, in which case it raises the abort flag and records a timeout.
-__device__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
-                          int where) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *abort_flag = 1;
-        report_status(status, GPTQ_ERR_TIMEOUT, where);
-        return false;
-      }
-    }
-  }
-}
-
-// Time-limited wait that ignores the abort flag (used to drain copies in flight after an abort).
-__device__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return;
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Shared-memory matrix descriptor, MN-major, 128-byte swizzle: 64-element rows of 128 B along the
-// M/N dimension, 8 rows (K) per 1024-byte swizzle atom.  LBO = byte stride between 64-element
-// chunks along M/N, SBO = byte stride between 8-row groups along K.
-__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t desc = 0;
-  desc |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  desc |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  desc |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  desc |= (uint64_t)1 << 46;  // descriptor version for sm_100
-  desc |= (uint64_t)2 << 61;  // SWIZZLE_128B
-  return desc;
-}
+using namespace tc;
 
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -177,30 +97,6 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // unit -> (tile row block bi, tile column block bj, split s)
@@ -252,10 +148,7 @@ __global__ void __launch_bounds__(THREADS, 1) hessian_tc_kernel(const __grid_con
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(tmem_slot, TMEM_COLS);
   }
   tc_fence_before();
   __syncthreads();
@@ -324,8 +217,8 @@ __global__ void __launch_bounds__(THREADS, 1) hessian_tc_kernel(const __grid_con
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               // 16 tokens = 2 swizzle atoms = 2048 bytes further along K
-              const uint64_t ad = sdesc_mn_sw128(A + kk * 2048, CHUNK_BYTES, 1024);
-              const uint64_t bd = sdesc_mn_sw128(B + kk * 2048, CHUNK_BYTES, 1024);
+              const uint64_t ad = sdesc_sw128(A + kk * 2048, CHUNK_BYTES, 1024);
+              const uint64_t bd = sdesc_sw128(B + kk * 2048, CHUNK_BYTES, 1024);
               umma_f16(d_tmem, ad, bd, a.idesc, (c > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&empty[slot]);
@@ -411,8 +304,7 @@ __global__ void __launch_bounds__(THREADS, 1) hessian_tc_kernel(const __grid_con
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                 : "memory");
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -452,18 +344,6 @@ __global__ void hessian_tc_reduce_kernel(const float* __restrict__ partial, int 
   *dst = out;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 constexpr int kSmemBytes = STAGES * STAGE_BYTES + 1024 + 256;
 
 }  // namespace
@@ -482,7 +362,7 @@ int hessian_tc_launches(int64_t n_tokens, int64_t d) { return tc_plan(n_tokens, 
 
 gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d, float* H, float scale,
                               int32_t accumulate, int32_t* status, void* workspace, cudaStream_t stream) {
-  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tc::encode_fn();
   if (encode == nullptr) return GPTQ_ERR_CUDA;
   TcPlan p = tc_plan(n_tokens, d);
   CUtensorMap map;

@@ -1,6 +1,7 @@
 // Internal launchers of the GPTQ solver kernels (host side; not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -21,6 +22,27 @@ int hessian_tc_launches(int64_t n_tokens, int64_t d);
 gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d, float* H, float scale,
                               int32_t accumulate, int32_t* status, void* workspace, cudaStream_t stream);
 
+// fp32-accurate 128x128-tile products on the tensor cores (3xTF32), gemm_tf32x3.cu
+enum Tf32x3Kind { kGemmTrsm = 0, kGemmSyrk = 1, kGemmTrtriT = 2, kGemmTrtriY = 3, kGemmLazy = 4 };
+enum Tf32x3Epi { kEpiStore = 0, kEpiStoreNeg = 1, kEpiSub = 2, kEpiStoreT = 3 };
+struct Tf32x3Args {
+  int kind, epi, b_mn, tiles;  // what, epilogue, B operand MN-major, work units
+  int p, skip;                 // trsm / syrk: panel; syrk: leading output tiles left out
+  int g, D;                    // trtri levels: half size and count of 128-blocks
+  int i1, i2, k, tiles_n;      // lazy update: U rows [i1, i1 + k), output columns from i2, column tiles
+  int o_w, o_h;                // output extent (columns, rows)
+  uint32_t idesc;              // set by the launcher
+  int32_t* status;
+};
+// 2-D fp32 tensor map (rows x cols, row stride ld elements), boxes of 32 columns x box_rows rows,
+// 128-byte swizzle (32-byte granules for an MN-major operand); false when the base or the stride is
+// not 16-byte aligned
+bool tf32x3_map(CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld, int box_rows,
+                bool mn_operand = false);
+// A: box rows 128 (K-major); B: box rows 128 (K-major) or 32 (MN-major map); O: box rows 32
+gptq_status tf32x3_gemm_launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O, Tf32x3Args a,
+                               cudaStream_t stream, int reserve_sms = 0);
+
 // A2 + A3
 size_t prepare_blocked_workspace(int64_t d);
 // lookahead: factor the next diagonal block on a library-owned second stream (made once per device)
@@ -38,7 +60,7 @@ size_t quantize_workspace(int64_t m, int64_t d, int block_size);
 bool quantize_fused(int64_t m, int64_t d);  // one launch per layer (U resident in L2) rather than launches per block
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
-                            void* workspace, cudaStream_t stream);
+                            int32_t* status, void* workspace, cudaStream_t stream);
 
 // A7
 gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,

@@ -160,10 +160,11 @@ __device__ void block_mm(float* out, const float* A, const float* B, bool tb, in
 }
 
 // Factors the 128x128 diagonal block p and writes side[p] = L(p,p)^-1 (row-major, zeros above the
-// diagonal).  When p > 0 the block first receives its last update, P(p,p) - L(p,p-1) L(p,p-1)^T (the
-// trailing update of panel p-1 leaves this block out, so its factorisation can run alongside).
-// Runs as block 0 of the panel-(p-1) update launch; 256 threads, dynamic shared memory.
-__device__ void factor_block(const float* P, int d, int p, float* side, int32_t* status, float* sm) {
+// diagonal).  With `update` (p > 0) the block first receives its last update,
+// P(p,p) - L(p,p-1) L(p,p-1)^T, here (the trailing update of panel p-1 then leaves this block out, so
+// the factorisation can run alongside it); otherwise the block arrives fully updated.
+// One CTA of 256 threads, dynamic shared memory.
+__device__ void factor_block(const float* P, int d, int p, bool update, float* side, int32_t* status, float* sm) {
   float* A = sm;                  // [128][LDS]
   float* Li = sm + BB * LDS;      // [128][LDS]
   float* S = Li + BB * LDS;       // [128][LDS]: L(p, p-1), then scratch
@@ -179,7 +180,7 @@ __device__ void factor_block(const float* P, int d, int p, float* side, int32_t*
       const int i = e / BB, c = e % BB;
       const int gi = p0 + i, gc = p0 + c;
       va[q] = (gi < d && gc < d) ? ((c <= i) ? P[(size_t)gi * d + gc] : 0.0f) : ((i == c) ? 1.0f : 0.0f);
-      vs[q] = (p > 0 && gi < d && gc - BB < d) ? P[(size_t)gi * d + gc - BB] : 0.0f;
+      vs[q] = (update && gi < d && gc - BB < d) ? P[(size_t)gi * d + gc - BB] : 0.0f;
     }
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
@@ -190,7 +191,7 @@ __device__ void factor_block(const float* P, int d, int p, float* side, int32_t*
     }
   }
   __syncthreads();
-  if (p > 0) block_mm(A, S, S, true, BB, BB, BB, -1.0f, 1.0f);  // A -= L(p,p-1) L(p,p-1)^T
+  if (update) block_mm(A, S, S, true, BB, BB, BB, -1.0f, 1.0f);  // A -= L(p,p-1) L(p,p-1)^T
   for (int s = 0; s < BB / kSub; ++s) {
     float* Ass = A + s * kSub * LDS + s * kSub;
     if (threadIdx.x < 32) warp_factor_invert_128(Ass, Li + s * kSub * LDS + s * kSub, colv, rsm, d, p0 + s * kSub, status);
@@ -220,10 +221,10 @@ __device__ void factor_block(const float* P, int d, int p, float* side, int32_t*
 
 constexpr int kFactorSmem = (3 * BB * LDS + 3 * kSub) * sizeof(float);
 
-__global__ void __launch_bounds__(256) factor_kernel(const float* __restrict__ P, int d, int p, float* __restrict__ side,
-                                                     int32_t* status) {
+__global__ void __launch_bounds__(256) factor_kernel(const float* __restrict__ P, int d, int p, int update,
+                                                     float* __restrict__ side, int32_t* status) {
   extern __shared__ __align__(16) float fsm[];
-  factor_block(P, d, p, side, status, fsm);
+  factor_block(P, d, p, update != 0, side, status, fsm);
 }
 
 // ------------------------------------------------------------------ 128x128x128 tile products
@@ -422,6 +423,19 @@ LookAhead g_lookahead[64];
 
 }  // namespace
 
+namespace {
+// The 3xTF32 tensor-core path needs 16-byte aligned rows (d % 4 == 0) and bases; other orders run
+// the fp32 FMA tile kernel.
+struct TcMaps {
+  CUtensorMap p128, p32, p32mn, side128;
+};
+
+bool tc_maps(TcMaps& m, const float* P, const float* side, int d, int D) {
+  return tf32x3_map(&m.p128, P, d, d, d, 128) && tf32x3_map(&m.p32, P, d, d, d, 32) &&
+         tf32x3_map(&m.p32mn, P, d, d, d, 32, true) && tf32x3_map(&m.side128, side, (int64_t)D * BB, BB, BB, 128);
+}
+}  // namespace
+
 gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status, void* workspace,
                                    cudaStream_t s, bool lookahead) {
   const int d = (int)d64;
@@ -433,6 +447,8 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
   GPTQ_CUDA_TRY(cudaGetDevice(&dev));
   GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFactorSmem));
+  TcMaps maps;
+  const bool tc = tc_maps(maps, U, side, d, D);
   std::unique_lock<std::mutex> hold(g_lookahead_mu, std::defer_lock);
   LookAhead* la = nullptr;
   if (lookahead && dev < 64) {
@@ -449,44 +465,87 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
   GPTQ_LAUNCH_CHECK();
   reverse_damp_kernel<<<sms * 4, 256, 0, s>>>(H, d, lam, U);
   GPTQ_LAUNCH_CHECK();
-  factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, 0, side, status);
+  factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, 0, 0, side, status);
   GPTQ_LAUNCH_CHECK();
   TileArgs ta{U, side, d, D, 0, 0, 1};
+  Tf32x3Args g{};
+  g.D = D;
+  g.o_w = d;
+  g.o_h = d;
+  g.status = status;
+  gptq_status st = GPTQ_OK;
   for (int p = 0; p + 1 < D; ++p) {
     const int below = D - p - 1;
-    ta.p = p;
-    tile_gemm_kernel<kTrsm><<<below, 256, 0, s>>>(ta);
-    GPTQ_LAUNCH_CHECK();
-    cudaStream_t fs = s;
+    const int tri = below * (below + 1) / 2;
+    // trsm(p)
+    if (tc) {
+      g.kind = kGemmTrsm, g.epi = kEpiStore, g.b_mn = 0, g.tiles = below, g.p = p, g.skip = 0;
+      if ((st = tf32x3_gemm_launch(maps.p128, maps.side128, maps.p32, g, s)) != GPTQ_OK) return st;
+    } else {
+      ta.p = p;
+      tile_gemm_kernel<kTrsm><<<below, 256, 0, s>>>(ta);
+      GPTQ_LAUNCH_CHECK();
+    }
+    // factor(p+1) and the trailing update of panel p.  On the tensor-core path the next diagonal
+    // block gets its update as a one-tile product first, and the trailing update leaves one SM free
+    // for that chain; on the fp32 path the factorisation does the diagonal update itself.
+    cudaStream_t fs = (la != nullptr) ? la->side : s;
     if (la != nullptr) {
       GPTQ_CUDA_TRY(cudaEventRecord(la->fork, s));
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
-      fs = la->side;
-      factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, side, status);
-      GPTQ_LAUNCH_CHECK();
-      GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
     }
-    const int tiles = below * (below + 1) / 2 - 1;
-    if (tiles > 0) {
-      tile_gemm_kernel<kSyrk><<<tiles, 256, 0, s>>>(ta);
-      GPTQ_LAUNCH_CHECK();
-    }
-    if (la != nullptr) {
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+    if (tc) {
+      if (la != nullptr) {
+        g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = 1, g.p = p, g.skip = 0;
+        if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, fs)) != GPTQ_OK) return st;
+        factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, 0, side, status);
+        GPTQ_LAUNCH_CHECK();
+        GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
+        g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = tri - 1, g.p = p, g.skip = 1;
+        if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, s, 1)) != GPTQ_OK) return st;
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+      } else {
+        g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = tri, g.p = p, g.skip = 0;
+        if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, s)) != GPTQ_OK) return st;
+        factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, 0, side, status);
+        GPTQ_LAUNCH_CHECK();
+      }
     } else {
-      factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, side, status);
-      GPTQ_LAUNCH_CHECK();
+      if (la != nullptr) {
+        factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, 1, side, status);
+        GPTQ_LAUNCH_CHECK();
+        GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
+      }
+      if (tri > 1) {
+        ta.p = p;
+        tile_gemm_kernel<kSyrk><<<tri - 1, 256, 0, s>>>(ta);
+        GPTQ_LAUNCH_CHECK();
+      }
+      if (la != nullptr) {
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+      } else {
+        factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, 1, side, status);
+        GPTQ_LAUNCH_CHECK();
+      }
     }
   }
   leaf_copy_kernel<<<D, 256, 0, s>>>(U, d, side);
   GPTQ_LAUNCH_CHECK();
-  for (int g = 1; g < D; g *= 2) {
-    const int pairs = (D + 2 * g - 1) / (2 * g);
-    ta.g = g;
-    tile_gemm_kernel<kTrtriT><<<pairs * g * g, 256, 0, s>>>(ta);
-    GPTQ_LAUNCH_CHECK();
-    tile_gemm_kernel<kTrtriY><<<pairs * g * g, 256, 0, s>>>(ta);
-    GPTQ_LAUNCH_CHECK();
+  for (int gl = 1; gl < D; gl *= 2) {
+    const int pairs = (D + 2 * gl - 1) / (2 * gl);
+    if (tc) {
+      g.g = gl, g.tiles = pairs * gl * gl, g.skip = 0, g.p = 0;
+      g.kind = kGemmTrtriT, g.epi = kEpiStoreT, g.b_mn = 1;
+      if ((st = tf32x3_gemm_launch(maps.p128, maps.p32mn, maps.p32, g, s)) != GPTQ_OK) return st;
+      g.kind = kGemmTrtriY, g.epi = kEpiStoreNeg, g.b_mn = 0;
+      if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, s)) != GPTQ_OK) return st;
+    } else {
+      ta.g = gl;
+      tile_gemm_kernel<kTrtriT><<<pairs * gl * gl, 256, 0, s>>>(ta);
+      GPTQ_LAUNCH_CHECK();
+      tile_gemm_kernel<kTrtriY><<<pairs * gl * gl, 256, 0, s>>>(ta);
+      GPTQ_LAUNCH_CHECK();
+    }
   }
   rotate_kernel<<<sms * 4, 256, 0, s>>>(U, d);
   GPTQ_LAUNCH_CHECK();

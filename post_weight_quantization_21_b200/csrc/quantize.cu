@@ -441,21 +441,45 @@ void launch_convert(const void* W, int64_t m, int d, int bits, int gs, float* ww
   convert_rowgrid_kernel<T><<<grid, 256, 0, s>>>(static_cast<const T*>(W), m, d, bits, gs, ww, sc, z);
 }
 
+// Per-block launches: the column loop of block [i1, i1 + B) for all rows, then the lazy update of the
+// trailing columns, on the tensor cores (3xTF32) unless `fma` asks for the fp32 FMA tile kernel or the
+// buffers are not 16-byte aligned for TMA.
 template <int NS>
 gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, int gs, uint8_t* codes,
-                       float* scales, int32_t* zeros, float* err, cudaStream_t s) {
+                       float* scales, int32_t* zeros, float* err, bool fma, int32_t* status, cudaStream_t s) {
   constexpr int B = 32 * NS;
   const int smem = (B * B + B) * sizeof(float);
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid_rows = (int)((m + kRowsPerCta - 1) / kRowsPerCta);
+  CUtensorMap mErr, mU, mW;
+  const bool tc = !fma && status != nullptr && tf32x3_map(&mErr, err, m, B, B, 128) &&
+                  tf32x3_map(&mU, U, d, d, d, 32, true) && tf32x3_map(&mW, ww, m, d, d, 32);
+  Tf32x3Args g{};
+  g.kind = kGemmLazy;
+  g.epi = kEpiSub;
+  g.b_mn = 1;
+  g.k = B;
+  g.o_w = d;
+  g.o_h = (int)m;
+  g.status = status;
+  const int tiles_m = (int)((m + 127) / 128);
   for (int i1 = 0; i1 < d; i1 += B) {
     colloop_kernel<NS><<<grid_rows, 256, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {
-      dim3 grid((unsigned)((m + 127) / 128), (rest + 127) / 128);
-      lazy_gemm_kernel<B><<<grid, 256, 0, s>>>(ww, m, d, i1, U, err);
-      GPTQ_LAUNCH_CHECK();
+      if (tc) {
+        g.i1 = i1;
+        g.i2 = i1 + B;
+        g.tiles_n = (rest + 127) / 128;
+        g.tiles = tiles_m * g.tiles_n;
+        const gptq_status st = tf32x3_gemm_launch(mErr, mU, mW, g, s);
+        if (st != GPTQ_OK) return st;
+      } else {
+        dim3 grid((unsigned)((m + 127) / 128), (rest + 127) / 128);
+        lazy_gemm_kernel<B><<<grid, 256, 0, s>>>(ww, m, d, i1, U, err);
+        GPTQ_LAUNCH_CHECK();
+      }
     }
   }
   return GPTQ_OK;
@@ -498,8 +522,9 @@ bool quantize_fused(int64_t m, int64_t d) { return d <= 4096 && m <= 2048; }
 
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d64, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
-                            void* workspace, cudaStream_t s) {
+                            int32_t* status, void* workspace, cudaStream_t s) {
   const int d = (int)d64;
+  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), s));
   char* ws = static_cast<char*>(workspace);
   float* ww = reinterpret_cast<float*>(ws);
   float* err = reinterpret_cast<float*>(ws + align_up((size_t)m * d * sizeof(float), 256));
@@ -518,10 +543,11 @@ gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d
     default: return GPTQ_ERR_ARG;
   }
   GPTQ_LAUNCH_CHECK();
+  const bool fma = (cfg.flags & GPTQ_FLAG_FP32_FMA) != 0;
   switch (cfg.block_size) {
-    case 32: return run_blocks<1>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, s);
-    case 64: return run_blocks<2>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, s);
-    case 128: return run_blocks<4>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, s);
+    case 32: return run_blocks<1>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s);
+    case 64: return run_blocks<2>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s);
+    case 128: return run_blocks<4>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s);
     default: return GPTQ_ERR_ARG;
   }
 }

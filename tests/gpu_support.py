@@ -41,7 +41,8 @@ def prepare(H: torch.Tensor, damp: float = 0.01, expect_ok: bool = True):
     return U, code, detail
 
 
-def quantize(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int, block_size: int, rows=None):
+def quantize(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int, block_size: int, rows=None,
+             flags: int = 0):
     """Codes, scales, zeros of the whole layer (of ``rows`` only when given) as int64/fp32 host arrays."""
     m, d = W.shape
     n_groups = 1 if group_size == 0 else d // group_size
@@ -50,8 +51,10 @@ def quantize(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int, block
     zeros = torch.empty(m, n_groups, dtype=torch.int32, device=W.device)
     ws = torch.empty(g.gptq_quantize_workspace_size(m, d, bits, group_size, block_size), dtype=torch.uint8,
                      device=W.device)
-    g.gptq_quantize_layer(W, U, codes, scales, zeros, ws, bits, group_size, block_size)
-    torch.cuda.synchronize()
+    st = torch.zeros(4, dtype=torch.int32, device=W.device)
+    g.gptq_quantize_layer(W, U, codes, scales, zeros, st, ws, bits, group_size, block_size, flags)
+    code, detail = g.gptq_read_status(st)
+    assert code == g.GPTQ_OK, (code, detail)
     if rows is not None:
         idx = torch.as_tensor(rows, device=W.device)
         codes, scales, zeros = codes[idx], scales[idx], zeros[idx]

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(g.ABI_FUNCTIONS)
-    assert lib.gptq_abi_version() == 1
+    assert lib.gptq_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -58,18 +58,26 @@ def test_workspace_sizes(lib):
 def test_validation_rejects_bad_arguments_without_a_device(lib):
     cfg = g.QuantCfg(4, 0, 128, 0)
     fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
-    st = lib.gptq_quantize_layer(fake, 1, 8, 100, fake, ctypes.byref(cfg), fake, fake, fake, fake, 1 << 20, None)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 100, fake, ctypes.byref(cfg), fake, fake, fake, fake, fake, 1 << 20, None)
     assert st == g.GPTQ_ERR_ARG                               # d % 32 != 0
     bad = g.QuantCfg(5, 0, 128, 0)
-    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(bad), fake, fake, fake, fake, 1 << 20, None)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(bad), fake, fake, fake, fake, fake, 1 << 20, None)
     assert st == g.GPTQ_ERR_ARG                               # bits = 5
     act = g.QuantCfg(4, 0, 128, g.GPTQ_FLAG_ACT_ORDER)
-    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(act), fake, fake, fake, fake, 1 << 20, None)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(act), fake, fake, fake, fake, fake, 1 << 20, None)
     assert st == g.GPTQ_ERR_UNSUPPORTED
     grp = g.QuantCfg(4, 96, 128, 0)                           # 96 and 128 do not divide one another
-    st = lib.gptq_quantize_layer(fake, 1, 8, 384, fake, ctypes.byref(grp), fake, fake, fake, fake, 1 << 20, None)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 384, fake, ctypes.byref(grp), fake, fake, fake, fake, fake, 1 << 20, None)
     assert st == g.GPTQ_ERR_ARG
-    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(cfg), fake, fake, fake, None, 0, None)
+    unknown = g.QuantCfg(4, 0, 128, 4)                        # no such flag bit
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(unknown), fake, fake, fake, fake, fake, 1 << 20,
+                                 None)
+    assert st == g.GPTQ_ERR_ARG
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(cfg), fake, fake, fake, None, fake, 1 << 20, None)
+    assert st == g.GPTQ_ERR_ARG                               # no status word
+    fma = g.QuantCfg(4, 0, 128, g.GPTQ_FLAG_FP32_FMA)
+    assert lib.gptq_quantize_workspace_size(8, 128, ctypes.byref(fma)) > 0
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(cfg), fake, fake, fake, fake, None, 0, None)
     assert st == g.GPTQ_ERR_WORKSPACE
     assert lib.gptq_pack(fake, 4, 48, 3, fake, None) == g.GPTQ_ERR_ARG        # d % 32
     assert lib.gptq_pack(fake, 4, 64, 5, fake, None) == g.GPTQ_ERR_ARG        # bits

@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import oracle
+import post_weight_quantization_21_b200 as g
 from post_weight_quantization_21_b200 import workloads as wl
 
 import gpu_support as S
@@ -74,7 +75,8 @@ def test_hessian_full_size_opt125m_layer():
 
 
 # ------------------------------------------------------------------------------------------ A2 + A3
-@pytest.mark.parametrize("d", [1, 5, 31, 33, 64, 128, 200, 768, 1000, 1100, 1500, 2048, 4224])
+# above 1024 the blocked path: tensor-core tiles when d % 4 == 0 (1100, 1500, 2048, 4224), fp32 tiles else (1102)
+@pytest.mark.parametrize("d", [1, 5, 31, 33, 64, 128, 200, 768, 1000, 1100, 1102, 1500, 2048, 4224])
 def test_prepare_matches_oracle(d):
     n = max(4 * d, 64)
     X = _x(n, d, torch.float64, seed=d)
@@ -111,8 +113,14 @@ QUANT_CASES = [
     (64, 512, 4, 256, 128),
     (48, 384, 4, 64, 32),
     (1, 128, 4, 0, 128),
-    (2100, 256, 4, 0, 128),    # many rows: per-block launches with the all-rows lazy GEMM
-    (40, 4224, 3, 128, 128),   # wider than 4096: per-block launches instead of the fused kernel
+]
+
+# many rows or wider than 4096: per-block launches (column loop, then the all-rows lazy GEMM)
+PER_BLOCK_CASES = [
+    (2100, 256, 4, 0, 128),
+    (2500, 512, 3, 128, 128),
+    (2049, 256, 4, 0, 32),
+    (40, 4224, 3, 128, 128),
     (24, 4352, 4, 0, 64),
 ]
 
@@ -127,6 +135,19 @@ def test_quantize_matches_oracle_given_U(m, d, bits, gs, B):
     ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), bits, gs, B)
     gpu = S.quantize(W.to(S.dev()), torch.from_numpy(U32).to(S.dev()), bits, gs, B)
     S.compare_quantization(gpu, ref, gs, W.double().numpy(), H, label=f"{m}x{d} b{bits} g{gs} B{B}")
+
+
+@pytest.mark.parametrize("flags", [0, g.GPTQ_FLAG_FP32_FMA], ids=["tf32x3", "fp32fma"])
+@pytest.mark.parametrize("m,d,bits,gs,B", PER_BLOCK_CASES)
+def test_quantize_per_block_paths(m, d, bits, gs, B, flags):
+    X = _x(4 * d, d, torch.float64, seed=m * d + bits)
+    H = oracle.hessian(X.numpy())
+    U = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01))
+    U32 = np.ascontiguousarray(U, dtype=np.float32)
+    W = (torch.randn(m, d, generator=torch.Generator().manual_seed(d + m)) * 0.02).half()
+    ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), bits, gs, B)
+    gpu = S.quantize(W.to(S.dev()), torch.from_numpy(U32).to(S.dev()), bits, gs, B, flags=flags)
+    S.compare_quantization(gpu, ref, gs, W.double().numpy(), H, label=f"{m}x{d} b{bits} g{gs} B{B} f{flags}")
 
 
 def test_quantize_fp32_and_bf16_weights():
