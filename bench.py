@@ -58,6 +58,9 @@ def peaks():
 
 
 # fp32 FMA peak of the part: 148 SMs x 128 FMA lanes x 2 flops x clock (nominal max 1965 MHz)
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 / bf16 tensor throughput of the B200
+
+
 def fp32_peak_tflops(sm_mhz: float) -> float:
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
@@ -284,27 +287,37 @@ def main():
     h2d = W_h.numel() * W_h.element_size() + X_h.numel() * X_h.element_size()
     d2h = sum(t.numel() * t.element_size() for t in (out_p, out_s, out_z))
 
-    # roofline of each phase (algorithmic work per launch / measured time)
+    # roofline of each phase (algorithmic work per launch / measured time), against the pipe the
+    # library runs it on for this shape: bf16 tensor cores (Hessian), 3xTF32 tensor cores (block
+    # products of the blocked prepare, lazy block updates), or fp32 FMA units
     sm_mhz = clk["sm_mhz"] if clk else 1965.0
     long_region = total_ms > 1000.0
     bf16_peak = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
     fp32_peak = fp32_peak_tflops(1965.0)
+    tf32x3_peak = bf16_peak * TF32_PER_BF16 / 3.0   # three tf32 MMAs per fp32-accurate product
+    tc = g.gptq_tensor_core_phases(L.m, L.d, L.n_tokens, L.x_dtype, L.bits, L.group_size, L.block_size)
     h_flops = L.n_tokens * L.d * (L.d + 1)                 # symmetric half of 2 N d^2
     p_flops = 2.0 / 3.0 * L.d ** 3                          # Cholesky + triangular inverse
     q_flops = float(L.m) * L.d * L.d                        # column loop + lazy updates
     k_bytes = L.m * L.d * (1 + L.bits / 8)                  # pack: codes in, words out
+    p_peak, p_pipe = (tf32x3_peak, "tensor(3xtf32)") if tc & g.GPTQ_TC_PREPARE else (fp32_peak, "fp32 FMA")
+    q_peak, q_pipe = (tf32x3_peak, "tensor(3xtf32)") if tc & g.GPTQ_TC_LAZY else (fp32_peak, "fp32 FMA")
     phases = {
         "hessian": {"ms": phase_ms[0], "tflops": h_flops / phase_ms[0] / 1e9,
                     "frac": h_flops / phase_ms[0] / 1e9 / bf16_peak, "pipe": "tensor(bf16)"},
         "prepare": {"ms": phase_ms[1], "tflops": p_flops / phase_ms[1] / 1e9,
-                    "frac": p_flops / phase_ms[1] / 1e9 / fp32_peak, "pipe": "fp32 FMA"},
+                    "frac": p_flops / phase_ms[1] / 1e9 / p_peak, "pipe": p_pipe},
         "quantize": {"ms": phase_ms[2], "tflops": q_flops / phase_ms[2] / 1e9,
-                     "frac": q_flops / phase_ms[2] / 1e9 / fp32_peak, "pipe": "fp32 FMA"},
+                     "frac": q_flops / phase_ms[2] / 1e9 / q_peak, "pipe": q_pipe},
         "pack": {"ms": phase_ms[3], "gbs": k_bytes / phase_ms[3] / 1e6,
                  "frac": k_bytes / phase_ms[3] / 1e6 / pk["hbm_gbs"], "pipe": "hbm"},
     }
-    roof_ms = (h_flops / bf16_peak / 1e9 + p_flops / fp32_peak / 1e9 + q_flops / fp32_peak / 1e9
+    roof_ms = (h_flops / bf16_peak / 1e9 + p_flops / p_peak / 1e9 + q_flops / q_peak / 1e9
                + k_bytes / pk["hbm_gbs"] / 1e6)
+    # the same sum with prepare and quantize bounded by the fp32 FMA units (their roofline before
+    # the block products moved to the tensor cores)
+    roof_fp32_ms = (h_flops / bf16_peak / 1e9 + p_flops / fp32_peak / 1e9 + q_flops / fp32_peak / 1e9
+                    + k_bytes / pk["hbm_gbs"] / 1e6)
     h_tflops = h_flops / phase_ms[0] / 1e9
     roofline = {"bound": "tensor", "kernel": "hessian (A1)", "achieved": h_tflops, "peak": bf16_peak,
                 "unit": "TFLOP/s", "frac": h_tflops / bf16_peak,
@@ -319,6 +332,11 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches), "roofline": roofline, "phases": phases,
             "phase_roofline_ms": roof_ms, "end_to_end_roofline_frac": roof_ms / ms_per_step,
+            "peaks": {"bf16_tflops": bf16_peak, "tf32x3_tflops": tf32x3_peak, "fp32_fma_tflops": fp32_peak,
+                      "hbm_gbs": pk["hbm_gbs"],
+                      "note": "bf16 and HBM measured; tf32 = bf16 x 1.1/2.25 (nominal ratio) / 3 MMAs; fp32 FMA = "
+                              "148 SMs x 128 lanes x 2 x 1965 MHz"},
+            "end_to_end_roofline_frac_fp32_pipes": roof_fp32_ms / ms_per_step,
             "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         W64 = W_h.double().numpy()

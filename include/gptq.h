@@ -189,6 +189,21 @@ GPTQ_API int32_t gptq_abi_version(void);
  * all threads).  Host-side counter; reading it does not touch the device. */
 GPTQ_API uint64_t gptq_kernel_launches(void);
 
+/* Diagnostics: which phases run their block products on the tensor cores for this shape, as a bit
+ * mask (host only, no device access):
+ *   GPTQ_TC_HESSIAN  H = scale X^T X with tcgen05 kind::f16 (16-bit X, d >= 256, n_tokens >= 64);
+ *                    otherwise fp32 FMA tiles.
+ *   GPTQ_TC_PREPARE  the blocked factorisation's trsm / syrk / triangular-inverse tiles as 3xTF32
+ *                    (d > 1024 and d % 4 == 0); smaller orders run the one-launch fp32 kernel.
+ *   GPTQ_TC_LAZY     the lazy block updates as 3xTF32 (the per-block path: d > 4096 or m > 2048,
+ *                    and no GPTQ_FLAG_FP32_FMA); otherwise fp32 FMA.
+ * Returns -1 when the arguments are invalid. */
+#define GPTQ_TC_HESSIAN 1
+#define GPTQ_TC_PREPARE 2
+#define GPTQ_TC_LAZY 4
+GPTQ_API int32_t gptq_tensor_core_phases(int64_t m, int64_t d, int64_t n_tokens, int32_t x_dtype,
+                                         const gptq_quant_cfg* cfg);
+
 #ifdef __cplusplus
 }
 #endif

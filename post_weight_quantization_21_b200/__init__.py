@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "GPTQError", "lib", "gptq_hessian_accumulate", "gptq_hessian_workspace_size", "gptq_prepare_uinv",
     "gptq_prepare_workspace_size", "gptq_prepare_uinv_static", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
-    "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
+    "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "gptq_tensor_core_phases", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -32,6 +32,7 @@ GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
 GPTQ_BF16, GPTQ_FP16, GPTQ_FP32 = 0, 1, 2
 GPTQ_FLAG_ACT_ORDER = 1
 GPTQ_FLAG_FP32_FMA = 2
+GPTQ_TC_HESSIAN, GPTQ_TC_PREPARE, GPTQ_TC_LAZY = 1, 2, 4
 
 _DTYPES = {torch.bfloat16: GPTQ_BF16, torch.float16: GPTQ_FP16, torch.float32: GPTQ_FP32}
 
@@ -56,6 +57,7 @@ ABI_FUNCTIONS = {
     "gptq_status_string": (ctypes.c_char_p, [_i32]),
     "gptq_abi_version": (_i32, []),
     "gptq_kernel_launches": (ctypes.c_uint64, []),
+    "gptq_tensor_core_phases": (_i32, [_i64, _i64, _i64, _i32, ctypes.POINTER(QuantCfg)]),
 }
 
 _lib = None
@@ -180,6 +182,13 @@ def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None)
     _contig(codes, "codes"), _contig(packed, "packed")
     m, d = codes.shape
     _check(lib().gptq_pack(_ptr(codes), m, d, bits, _ptr(packed), _stream(stream)), "gptq_pack")
+
+
+def gptq_tensor_core_phases(m: int, d: int, n_tokens: int, x_dtype, bits: int, group_size: int = 0,
+                            block_size: int = 128, flags: int = 0) -> int:
+    """Bit mask of the phases whose block products run on the tensor cores (GPTQ_TC_*)."""
+    c = _cfg(bits, group_size, block_size, flags)
+    return int(lib().gptq_tensor_core_phases(m, d, n_tokens, _DTYPES[x_dtype], ctypes.byref(c)))
 
 
 def gptq_kernel_launches() -> int:

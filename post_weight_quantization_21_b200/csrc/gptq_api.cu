@@ -44,6 +44,16 @@ int32_t gptq_abi_version(void) { return GPTQ_ABI_VERSION; }
 
 uint64_t gptq_kernel_launches(void) { return gptq::g_launches.load(std::memory_order_relaxed); }
 
+int32_t gptq_tensor_core_phases(int64_t m, int64_t d, int64_t n_tokens, int32_t x_dtype, const gptq_quant_cfg* cfg) {
+  if (m <= 0 || d <= 0 || n_tokens < 0 || d > kMaxDim || !valid_dtype(x_dtype) || check_cfg(cfg, d) != GPTQ_OK)
+    return -1;
+  int32_t mask = 0;
+  if (gptq::hessian_tc_supported(n_tokens, d, x_dtype)) mask |= GPTQ_TC_HESSIAN;
+  if (gptq::prepare_uses_tensor_cores(d)) mask |= GPTQ_TC_PREPARE;
+  if (!gptq::quantize_fused(m, d) && !(cfg->flags & GPTQ_FLAG_FP32_FMA)) mask |= GPTQ_TC_LAZY;
+  return mask;
+}
+
 const char* gptq_status_string(int32_t status) {
   switch (status) {
     case GPTQ_OK: return "ok";

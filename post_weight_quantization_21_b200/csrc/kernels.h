@@ -49,6 +49,7 @@ size_t prepare_blocked_workspace(int64_t d);
 gptq_status prepare_blocked_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
                                    void* workspace, cudaStream_t stream, bool lookahead);
 size_t prepare_workspace(int64_t d);
+bool prepare_uses_tensor_cores(int64_t d);
 gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
                            void* workspace, cudaStream_t stream, bool lookahead = true);
 // same, with the scratch in a static device array (d <= GPTQ_PREPARE_STATIC_MAX_D)

@@ -454,6 +454,9 @@ constexpr size_t kSideOffset = 1024;
 // orders are dominated by dense block products and take the 128-block path (prepare_blocked.cu).
 constexpr int64_t kSmallOrder = 1024;
 
+// the blocked path's tile products go to the tensor cores when rows are 16-byte aligned
+bool prepare_uses_tensor_cores(int64_t d) { return d > kSmallOrder && d % 4 == 0; }
+
 size_t prepare_workspace(int64_t d) {
   if (d > kSmallOrder) return prepare_blocked_workspace(d);
   const int64_t D = (d + NB - 1) / NB;

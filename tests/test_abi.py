@@ -87,3 +87,14 @@ def test_validation_rejects_bad_arguments_without_a_device(lib):
     assert lib.gptq_prepare_uinv(fake, 16, 0.01, other, fake, None, 0, None) == g.GPTQ_ERR_WORKSPACE
     assert lib.gptq_prepare_uinv(fake, 16, -1.0, other, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG
     assert lib.gptq_prepare_uinv(fake, 16, 0.01, fake, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG  # H == U
+
+
+def test_tensor_core_phase_mask_without_a_device():
+    import torch
+    assert g.gptq_tensor_core_phases(768, 768, 262144, torch.bfloat16, 4) == g.GPTQ_TC_HESSIAN
+    all3 = g.GPTQ_TC_HESSIAN | g.GPTQ_TC_PREPARE | g.GPTQ_TC_LAZY
+    assert g.gptq_tensor_core_phases(4096, 4096, 262144, torch.bfloat16, 3, 128) == all3
+    assert g.gptq_tensor_core_phases(4096, 4096, 262144, torch.bfloat16, 3, 128,
+                                     flags=g.GPTQ_FLAG_FP32_FMA) == g.GPTQ_TC_HESSIAN | g.GPTQ_TC_PREPARE
+    assert g.gptq_tensor_core_phases(64, 4224, 256, torch.float32, 4) == g.GPTQ_TC_PREPARE | g.GPTQ_TC_LAZY
+    assert g.gptq_tensor_core_phases(64, 100, 256, torch.float32, 4) == -1   # block does not divide d
