@@ -178,48 +178,37 @@ __device__ __forceinline__ void zero(float acc[2][4]) {
 // LiT[m][y] = L^-1[y][m].  Lane i keeps row i of A; lane c keeps column c of the right-hand sides
 // of L Y = I.  Right-looking with an unscaled pivot column:
 //   A[i][x] -= A[i][k] A[x][k] / A[k][k],   R[x][c] -= A[x][k] R[k][c] / A[k][k]   (x > k)
-// then L^-1[i][c] = R[i][c] / sqrt(pivot_i).  The pivot column is shared through shared memory
-// (zeros at and above the pivot) and read four entries at a time.  pivot_base: reversed-order index
-// of the block's first column, for the failure report.
-__device__ void warp_factor_invert(const float (*A)[TS], float (*LiT)[TS], float* colv, float* rsm, int d,
-                                   int pivot_base, int32_t* status) {
+// then L^-1[i][c] = R[i][c] / sqrt(pivot_i).  Entry A[x][k] of the pivot column reaches every lane by
+// a shuffle from lane x.  pivot_base: reversed-order index of the block's first column, for the
+// failure report.
+__device__ void warp_factor_invert(const float (*A)[TS], float (*LiT)[TS], int d, int pivot_base, int32_t* status) {
   const int lane = threadIdx.x & 31;
-  float a[NB], rr[NB];
+  float a[NB], rr[NB], rs[NB];
 #pragma unroll
   for (int c = 0; c < NB; ++c) {
     a[c] = A[lane][c];
     rr[c] = (c == lane) ? 1.0f : 0.0f;
   }
+  int bad = -1;  // first non-positive pivot (the pivot is the same on every lane)
 #pragma unroll
   for (int k = 0; k < NB; ++k) {
-    float* cv = colv + (k & 1) * NB;
-    cv[lane] = (lane > k) ? a[k] : 0.0f;
     const float p = __shfl_sync(0xffffffffu, a[k], k);
-    __syncwarp();
     const float inv = __fdividef(1.0f, p);
+    rs[k] = rsqrtf(p);
+    if (bad < 0 && !(p > 0.0f && isfinite(p)) && pivot_base + k < d) bad = k;
     const float li = a[k] * inv;
     const float t = rr[k] * inv;
-    if (lane == 0) {
-      rsm[k] = rsqrtf(p);
-      if (!(p > 0.0f && isfinite(p)) && pivot_base + k < d) report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
-    }
 #pragma unroll
-    for (int x4 = (k + 1) & ~3; x4 < NB; x4 += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(cv + x4);
-      a[x4 + 0] = fmaf(-li, v.x, a[x4 + 0]);
-      a[x4 + 1] = fmaf(-li, v.y, a[x4 + 1]);
-      a[x4 + 2] = fmaf(-li, v.z, a[x4 + 2]);
-      a[x4 + 3] = fmaf(-li, v.w, a[x4 + 3]);
-      rr[x4 + 0] = fmaf(-v.x, t, rr[x4 + 0]);
-      rr[x4 + 1] = fmaf(-v.y, t, rr[x4 + 1]);
-      rr[x4 + 2] = fmaf(-v.z, t, rr[x4 + 2]);
-      rr[x4 + 3] = fmaf(-v.w, t, rr[x4 + 3]);
+    for (int x = k + 1; x < NB; ++x) {
+      const float v = __shfl_sync(0xffffffffu, a[k], x);  // A[x][k]
+      a[x] = fmaf(-li, v, a[x]);
+      rr[x] = fmaf(-v, t, rr[x]);
     }
   }
-  __syncwarp();
+  if (lane == 0 && bad >= 0) report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + bad));
   // column `lane` of L^-1 is row `lane` of LiT
 #pragma unroll
-  for (int i = 0; i < NB; ++i) LiT[lane][i] = (i >= lane) ? rr[i] * rsm[i] : 0.0f;
+  for (int i = 0; i < NB; ++i) LiT[lane][i] = (i >= lane) ? rr[i] * rs[i] : 0.0f;
   __syncwarp();
 }
 
@@ -229,7 +218,6 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
   __shared__ __align__(16) float S2[NB][TS];
   __shared__ __align__(16) float S3[NB][TS];
   __shared__ __align__(16) float S4[NB][TS];
-  __shared__ __align__(16) float colv[3 * NB];  // two pivot-column buffers + 1/sqrt(pivot)
   const int tid = threadIdx.x;
   const int ty = tid >> 3, tx = tid & 7;
   const int d = a.d, D = a.D;
@@ -316,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
           for (int e = tid; e < NB * NB; e += kThreads) S3[e & 31][e >> 5] = S1[e >> 5][e & 31];
         }
         __syncthreads();
-        if (tid < 32) warp_factor_invert(S0, S4, colv, colv + 2 * NB, d, j * NB, a.status);
+        if (tid < 32) warp_factor_invert(S0, S4, d, j * NB, a.status);
         __syncthreads();
         if (r == j) {
           float* out = a.side + (size_t)j * NB * NB;  // natural layout: out[y][m] = S4[m][y]

@@ -62,99 +62,95 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const fl
 
 // ------------------------------------------------------------------ panel factorisation
 // One warp factors a 32x32 block (lower part, stride LDS) and writes its inverse, natural layout,
-// into Li (stride LDS): lane i keeps row i of A, lane c keeps column c of the right-hand sides of
-// L Y = I; right-looking with an unscaled pivot column.
-__device__ void warp_factor_invert_128(const float* A, float* Li, float* colv, float* rsm, int d, int pivot_base,
-                                       int32_t* status) {
+// into Li (stride LDS): lane i keeps row i of A and column i of the right-hand sides of L Y = I;
+// right-looking with an unscaled pivot column, column k reaching every lane by shuffles.
+__device__ void warp_factor_invert_128(const float* A, float* Li, int d, int pivot_base, int32_t* status) {
   const int lane = threadIdx.x & 31;
-  float a[kSub], rr[kSub];
+  float a[kSub], rr[kSub], rs[kSub];
 #pragma unroll
   for (int c = 0; c < kSub; ++c) {
     a[c] = A[lane * LDS + c];
     rr[c] = (c == lane) ? 1.0f : 0.0f;
   }
+  int bad = -1;  // first non-positive pivot (the pivot is the same on every lane)
 #pragma unroll
   for (int k = 0; k < kSub; ++k) {
-    float* cv = colv + (k & 1) * kSub;
-    cv[lane] = (lane > k) ? a[k] : 0.0f;
     const float p = __shfl_sync(0xffffffffu, a[k], k);
-    __syncwarp();
     const float inv = __fdividef(1.0f, p);
+    rs[k] = rsqrtf(p);
+    if (bad < 0 && !(p > 0.0f && isfinite(p)) && pivot_base + k < d) bad = k;
     const float li = a[k] * inv;
     const float t = rr[k] * inv;
-    if (lane == 0) {
-      rsm[k] = rsqrtf(p);
-      if (!(p > 0.0f && isfinite(p)) && pivot_base + k < d) report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + k));
-    }
 #pragma unroll
-    for (int x4 = (k + 1) & ~3; x4 < kSub; x4 += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(cv + x4);
-      a[x4 + 0] = fmaf(-li, v.x, a[x4 + 0]);
-      a[x4 + 1] = fmaf(-li, v.y, a[x4 + 1]);
-      a[x4 + 2] = fmaf(-li, v.z, a[x4 + 2]);
-      a[x4 + 3] = fmaf(-li, v.w, a[x4 + 3]);
-      rr[x4 + 0] = fmaf(-v.x, t, rr[x4 + 0]);
-      rr[x4 + 1] = fmaf(-v.y, t, rr[x4 + 1]);
-      rr[x4 + 2] = fmaf(-v.z, t, rr[x4 + 2]);
-      rr[x4 + 3] = fmaf(-v.w, t, rr[x4 + 3]);
+    for (int x = k + 1; x < kSub; ++x) {
+      const float v = __shfl_sync(0xffffffffu, a[k], x);  // A[x][k]
+      a[x] = fmaf(-li, v, a[x]);
+      rr[x] = fmaf(-v, t, rr[x]);
     }
   }
-  __syncwarp();
+  if (lane == 0 && bad >= 0) report_status(status, GPTQ_ERR_NOT_PD, d - 1 - (pivot_base + bad));
   // lane holds column `lane` of the right-hand sides: Linv[i][lane] = rr[i] / sqrt(pivot_i)
 #pragma unroll
-  for (int i = 0; i < kSub; ++i) Li[i * LDS + lane] = (i >= lane) ? rr[i] * rsm[i] : 0.0f;
+  for (int i = 0; i < kSub; ++i) Li[i * LDS + lane] = (i >= lane) ? rr[i] * rs[i] : 0.0f;
   __syncwarp();
 }
 
 // out (M x N, stride LDS) = beta * out + alpha * sum_{k<K} A[m][k] * B(k, n), by all 256 threads;
-// M and N multiples of 32, at most 128.  B(k, n) = B[n][k] (tb) or B[k][n] (!tb).  The output is cut
-// into 32x32 warp tiles; lane (mi, ni) = (lane / 8, lane % 8) of a warp owns rows mi + 4i and
-// columns ni + 8j of its tile, which keeps the shared-memory reads free of bank conflicts with the
-// row stride LDS.  Products are kept in registers and stored after a barrier, so out may alias the
-// inputs.  beta is 0 or 1.
-__device__ void block_mm(float* out, const float* A, const float* B, bool tb, int M, int N, int K, float alpha,
-                         float beta) {
+// M, N multiples of 16 (at most 128), K a multiple of 4; out must not overlap A or B.
+// B(k, n) = B[n][k] (TB) or B[k][n] (!TB).  The output is cut into 16x16 warp tiles dealt
+// round-robin to the 8 warps, so small products still use every warp; lane (mi, ni) = (lane / 4,
+// lane % 4) owns rows mi + 8i and columns ni + 4j of its tile.  A (and B when TB) is read as float4
+// along k; with the row stride LDS = 132 the rows of one load fall in distinct bank groups.  The
+// pass loop stays rolled: these products run once each per launch, so a compact body keeps the
+// kernel inside the instruction cache.  Ends with a barrier.  beta is 0 or 1.
+template <bool TB>
+__device__ void block_mm(float* out, const float* A, const float* B, int M, int N, int K, float alpha, float beta) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mi = lane >> 3, ni = lane & 7;
-  const int wn = N / 32, n_wt = (M / 32) * wn;
-  float r[2][8][4];
+  const int mi = lane >> 2, ni = lane & 3;
+  const int wn = N / 16, n_wt = (M / 16) * wn;
+#pragma unroll 1
+  for (int wt = warp; wt < n_wt; wt += 8) {
+    float r[2][4];
 #pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int wt = warp + pass * 8;
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+      for (int j = 0; j < 4; ++j) r[i][j] = 0.0f;
+    const float* a = A + ((wt / wn) * 16 + mi) * LDS;
+    const int n0 = (wt % wn) * 16 + ni;
+#pragma unroll 2
+    for (int k = 0; k < K; k += 4) {
+      float4 av[2], bv[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) r[pass][i][j] = 0.0f;
-    if (wt < n_wt) {
-      const float* a = A + ((wt / wn) * 32 + mi) * LDS;
-      const int n0 = (wt % wn) * 32 + ni;
-      for (int k = 0; k < K; ++k) {
-        float av[8], bv[4];
+      for (int i = 0; i < 2; ++i) av[i] = *reinterpret_cast<const float4*>(a + 8 * i * LDS + k);
+      if (TB) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) av[i] = a[4 * i * LDS + k];
+        for (int j = 0; j < 4; ++j) bv[j] = *reinterpret_cast<const float4*>(B + (n0 + 4 * j) * LDS + k);
+      } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) bv[j] = tb ? B[(n0 + 8 * j) * LDS + k] : B[k * LDS + n0 + 8 * j];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) r[pass][i][j] = fmaf(av[i], bv[j], r[pass][i][j]);
+        for (int j = 0; j < 4; ++j)
+          bv[j] = make_float4(B[k * LDS + n0 + 4 * j], B[(k + 1) * LDS + n0 + 4 * j], B[(k + 2) * LDS + n0 + 4 * j],
+                              B[(k + 3) * LDS + n0 + 4 * j]);
       }
-    }
-  }
-  __syncthreads();
 #pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int wt = warp + pass * 8;
-    if (wt < n_wt) {
-      float* o = out + ((wt / wn) * 32 + mi) * LDS + (wt % wn) * 32 + ni;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float* e = o + 4 * i * LDS + 8 * j;
-          *e = (beta != 0.0f ? *e : 0.0f) + alpha * r[pass][i][j];
+          float acc = r[i][j];
+          acc = fmaf(av[i].x, bv[j].x, acc);
+          acc = fmaf(av[i].y, bv[j].y, acc);
+          acc = fmaf(av[i].z, bv[j].z, acc);
+          acc = fmaf(av[i].w, bv[j].w, acc);
+          r[i][j] = acc;
         }
     }
+    float* o = out + ((wt / wn) * 16 + mi) * LDS + (wt % wn) * 16 + ni;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float* e = o + 8 * i * LDS + 4 * j;
+        *e = (beta != 0.0f ? *e : 0.0f) + alpha * r[i][j];
+      }
   }
   __syncthreads();
 }
@@ -168,9 +164,32 @@ __device__ void factor_block(const float* P, int d, int p, bool update, float* s
   float* A = sm;                  // [128][LDS]
   float* Li = sm + BB * LDS;      // [128][LDS]
   float* S = Li + BB * LDS;       // [128][LDS]: L(p, p-1), then scratch
-  float* colv = S + BB * LDS;     // 2 x 32
-  float* rsm = colv + 2 * kSub;   // 32
   const int p0 = p * BB;
+  if (!update && d % 4 == 0) {
+    // 16-byte rows: one batch of 16 float4 loads per thread; the upper part and rows / columns past
+    // the order read as the identity
+    float4 va[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = threadIdx.x + q * 256;
+      const int i = e / (BB / 4), c = (e % (BB / 4)) * 4;
+      const int gi = p0 + i, gc = p0 + c;
+      va[q] = (gi < d && gc < d) ? *reinterpret_cast<const float4*>(P + (size_t)gi * d + gc) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = threadIdx.x + q * 256;
+      const int i = e / (BB / 4), c = (e % (BB / 4)) * 4;
+      const bool in = p0 + i < d;
+      float x[4] = {va[q].x, va[q].y, va[q].z, va[q].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool col_in = in && p0 + c + u < d;
+        A[i * LDS + c + u] = col_in ? ((c + u <= i) ? x[u] : 0.0f) : ((i == c + u) ? 1.0f : 0.0f);
+      }
+      *reinterpret_cast<float4*>(Li + i * LDS + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else
   // batched loads: every thread issues its 16 loads before storing
   for (int base = 0; base < BB * BB; base += 16 * 256) {
     float va[16], vs[16];
@@ -191,37 +210,47 @@ __device__ void factor_block(const float* P, int d, int p, bool update, float* s
     }
   }
   __syncthreads();
-  if (update) block_mm(A, S, S, true, BB, BB, BB, -1.0f, 1.0f);  // A -= L(p,p-1) L(p,p-1)^T
+  if (update) block_mm<true>(A, S, S, BB, BB, BB, -1.0f, 1.0f);  // A -= L(p,p-1) L(p,p-1)^T (S is free after)
+#pragma unroll 1
   for (int s = 0; s < BB / kSub; ++s) {
     float* Ass = A + s * kSub * LDS + s * kSub;
-    if (threadIdx.x < 32) warp_factor_invert_128(Ass, Li + s * kSub * LDS + s * kSub, colv, rsm, d, p0 + s * kSub, status);
+    if (threadIdx.x < 32) warp_factor_invert_128(Ass, Li + s * kSub * LDS + s * kSub, d, p0 + s * kSub, status);
     __syncthreads();
     const int rest = BB - (s + 1) * kSub;
     if (rest > 0) {
       float* Ats = A + (s + 1) * kSub * LDS + s * kSub;
-      block_mm(Ats, Ats, Li + s * kSub * LDS + s * kSub, true, rest, kSub, kSub, 1.0f, 0.0f);  // L(t, s)
+      float* Sts = S + (s + 1) * kSub * LDS + s * kSub;
+      block_mm<true>(Sts, Ats, Li + s * kSub * LDS + s * kSub, rest, kSub, kSub, 1.0f, 0.0f);  // L(t, s), into S
+      for (int e = threadIdx.x; e < rest * kSub / 4; e += blockDim.x) {  // ... and back into A
+        const int r = e / (kSub / 4), c = (e % (kSub / 4)) * 4;
+        *reinterpret_cast<float4*>(Ats + r * LDS + c) = *reinterpret_cast<const float4*>(Sts + r * LDS + c);
+      }
+      __syncthreads();
       float* Atr = A + (s + 1) * kSub * LDS + (s + 1) * kSub;
-      block_mm(Atr, Ats, Ats, true, rest, rest, kSub, -1.0f, 1.0f);  // trailing part of the block
+      block_mm<true>(Atr, Sts, Sts, rest, rest, kSub, -1.0f, 1.0f);  // trailing part of the block
     }
   }
   // [[A,0],[C,B]]^-1 = [[A^-1, 0], [-B^-1 C A^-1, B^-1]], 32 -> 64 -> 128
+#pragma unroll 1
   for (int h = kSub; h < BB; h *= 2) {
+#pragma unroll 1
     for (int a0 = 0; a0 < BB; a0 += 2 * h) {
       const int b0 = a0 + h;
-      block_mm(S, A + b0 * LDS + a0, Li + a0 * LDS + a0, false, h, h, h, 1.0f, 0.0f);
-      block_mm(Li + b0 * LDS + a0, Li + b0 * LDS + b0, S, false, h, h, h, -1.0f, 0.0f);
+      block_mm<false>(S, A + b0 * LDS + a0, Li + a0 * LDS + a0, h, h, h, 1.0f, 0.0f);
+      block_mm<false>(Li + b0 * LDS + a0, Li + b0 * LDS + b0, S, h, h, h, -1.0f, 0.0f);
     }
   }
-  float* out = side + (size_t)p * BB * BB;
-  for (int e = threadIdx.x; e < BB * BB; e += blockDim.x) {
-    const int i = e / BB, c = e % BB;
-    out[e] = (c <= i) ? Li[i * LDS + c] : 0.0f;
+  float4* out = reinterpret_cast<float4*>(side + (size_t)p * BB * BB);
+  for (int e = threadIdx.x; e < BB * BB / 4; e += blockDim.x) {
+    const int i = e / (BB / 4), c = (e % (BB / 4)) * 4;
+    const float4 l = *reinterpret_cast<const float4*>(Li + i * LDS + c);
+    out[e] = make_float4(c <= i ? l.x : 0.f, c + 1 <= i ? l.y : 0.f, c + 2 <= i ? l.z : 0.f, c + 3 <= i ? l.w : 0.f);
   }
 }
 
-constexpr int kFactorSmem = (3 * BB * LDS + 3 * kSub) * sizeof(float);
+constexpr int kFactorSmem = 3 * BB * LDS * sizeof(float);
 
-__global__ void __launch_bounds__(256) factor_kernel(const float* __restrict__ P, int d, int p, int update,
+__global__ void __launch_bounds__(256, 1) factor_kernel(const float* __restrict__ P, int d, int p, int update,
                                                      float* __restrict__ side, int32_t* status) {
   extern __shared__ __align__(16) float fsm[];
   factor_block(P, d, p, update != 0, side, status, fsm);

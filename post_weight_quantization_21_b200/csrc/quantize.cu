@@ -166,41 +166,135 @@ __device__ __forceinline__ void load_u_block(float* Us, float* invd, const float
   }
 }
 
-// Column loop over block [i1, i1 + 32*NS) for 8 rows per CTA (per-block launch path).
-template <int NS>
-__global__ void __launch_bounds__(256) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+
+// Column loop over block [i1, i1 + B) on the per-block launch path, 32 rows per CTA of 4 warps.
+// Four lanes (a quad) share a row: lane `sub` of the quad holds the C = B/4 consecutive columns
+// i1 + sub*C .. i1 + sub*C + C-1 in registers.  At block column i the owner lane (sub = i / C)
+// rounds its column, updates its own next column straight away (its chain stays in its registers
+// for C steps), and the error reaches the quad with one shuffle; each lane then applies it to its
+// columns after i.  The rounding runs once per warp instruction for 8 rows, so a row-step costs a
+// few warp instructions instead of a whole warp's.  The raw U block (B x B) sits in shared memory
+// with each row's four C-column chunks 16 bytes apart, so the quad's float4 reads of a row fall in
+// distinct bank groups; err * U[i, j] with err = delta / U_ii is the page's update.
+template <int C>
+__global__ void __launch_bounds__(128) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
                                                       const float* __restrict__ U, int bits,
                                                       int group_size, uint8_t* __restrict__ codes,
                                                       float* __restrict__ scales,
                                                       int32_t* __restrict__ zeros,
                                                       float* __restrict__ err_out) {
-  constexpr int B = 32 * NS;
-  extern __shared__ float sm[];
-  float* Us = sm;
-  float* invd = sm + B * B;
-  load_u_block<B>(Us, invd, U, d, i1);
-  __syncthreads();
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
-  if (row >= m) return;
-  float* wr = w + row * d;
-  float v[NS];
-#pragma unroll
-  for (int s = 0; s < NS; ++s) v[s] = wr[i1 + lane * NS + s];
-  const float maxq = (float)((1 << bits) - 1);
-  const int n_groups = group_size ? d / group_size : 1;
-  float scale, zero;
-  grid_at_block(row, i1, group_size, n_groups, scales, zeros, scale, zero);
-  float rscale = __frcp_rn(scale);
-  uint32_t code_reg[NS];
-  float err_reg[NS];
-  column_loop<NS>(v, Us, invd, i1, group_size, n_groups, maxq, scale, zero, rscale, wr, row, scales, zeros,
-                  code_reg, err_reg);
-#pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    codes[row * d + i1 + lane * NS + s] = (uint8_t)code_reg[s];
-    err_out[row * B + lane * NS + s] = err_reg[s];
+  constexpr int B = 4 * C;
+  constexpr int CS = C + 4;   // chunk stride
+  constexpr int RS = 4 * CS;  // row stride
+  extern __shared__ __align__(16) float sm[];
+  float* Ub = sm;             // U[i1 + r][i1 + q*C + t] at Ub[r*RS + q*CS + t]
+  float* invd = sm + B * RS;  // 1 / U_ii
+  for (int e = threadIdx.x; e < B * B / 4; e += blockDim.x) {
+    const int r = e / (B / 4), c = (e % (B / 4)) * 4;
+    cp_async16(Ub + r * RS + (c / C) * CS + c % C, U + (size_t)(i1 + r) * d + i1 + c);
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  if (threadIdx.x < B) invd[threadIdx.x] = 1.0f / U[(size_t)(i1 + threadIdx.x) * d + i1 + threadIdx.x];
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane & 3;
+  const int qbase = lane & ~3;
+  const int64_t row = ((int64_t)blockIdx.x * (blockDim.x / 32) + warp) * 8 + (lane >> 2);
+  const bool valid = row < m;  // lanes past the last row keep shuffling with zeros
+  const int n_groups = group_size ? d / group_size : 1;
+  float* wrow = w + (valid ? row : 0) * d;
+  float v[C];
+#pragma unroll
+  for (int q = 0; q < C / 4; ++q) {
+    const float4 x = valid ? *reinterpret_cast<const float4*>(wrow + i1 + sub * C + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[4 * q] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
+  }
+  const float maxq = (float)((1 << bits) - 1);
+  float scale = 1.0f, zero = 0.0f;
+  if (valid) grid_at_block(row, i1, group_size, n_groups, scales, zeros, scale, zero);
+  float rscale = __frcp_rn(scale);
+  uint32_t cw[C / 4];
+  float er[C];
+#pragma unroll
+  for (int q = 0; q < C / 4; ++q) cw[q] = 0u;
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+#pragma unroll 1
+  for (int o = 0; o < 4; ++o) {
+    const bool owner = (sub == o);
+#pragma unroll
+    for (int s = 0; s < C; ++s) {
+      const int i = o * C + s;  // block column
+      if (s == 0 && group_size != 0 && ((i1 + i) % group_size) == 0) {
+        // grid of the group starting here, from the current values of its columns
+        const int gend = i + group_size;  // block-local end (may pass the block)
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < C; ++t) {
+          const int c = sub * C + t;
+          if (c >= i && c < gend) {
+            mn = fminf(mn, v[t]);
+            mx = fmaxf(mx, v[t]);
+          }
+        }
+        if (valid)
+          for (int c = i1 + B + sub; c < i1 + gend; c += 4) {  // group wider than the rest of the block
+            const float x = wrow[c];
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        grid_from_range(mn, mx, maxq, scale, zero, rscale);
+        if (sub == 0 && valid) {
+          const int g = (i1 + i) / group_size;
+          scales[row * n_groups + g] = scale;
+          zeros[row * n_groups + g] = (int32_t)zero;
+        }
+      }
+      const float wi = v[s];  // the owner's column (other lanes compute and discard)
+      // code - zero, clamped to the grid; the quotient as an IEEE fp32 product with 1/scale
+      const float qz = fminf(fmaxf(rintf(__fmul_rn(wi, rscale)), -zero), maxq - zero);
+      const float delta = fmaf(-scale, qz, wi);  // w_i - dequantized value
+      const float err = delta * invd[i];
+      const float* urow = Ub + i * RS + sub * CS;
+      if (owner) {
+        cw[s >> 2] |= (uint32_t)(qz + zero) << (8 * (s & 3));
+        er[s] = err;
+        if (s + 1 < C) v[s + 1] = fmaf(-err, urow[s + 1], v[s + 1]);  // the owner's next column first
+      }
+      const float e = __shfl_sync(0xffffffffu, err, qbase | o);
+      // columns after i: every column of a lane past the owner, the owner's columns after s + 1
+      const float f_near = (sub > o) ? e : 0.0f;
+      const float f_far = (sub >= o) ? e : 0.0f;
+#pragma unroll
+      for (int q = 0; q < C / 4; ++q) {
+        const float4 u = reinterpret_cast<const float4*>(urow)[q];
+        v[4 * q + 0] = fmaf(4 * q + 0 <= s + 1 ? -f_near : -f_far, u.x, v[4 * q + 0]);
+        v[4 * q + 1] = fmaf(4 * q + 1 <= s + 1 ? -f_near : -f_far, u.y, v[4 * q + 1]);
+        v[4 * q + 2] = fmaf(4 * q + 2 <= s + 1 ? -f_near : -f_far, u.z, v[4 * q + 2]);
+        v[4 * q + 3] = fmaf(4 * q + 3 <= s + 1 ? -f_near : -f_far, u.w, v[4 * q + 3]);
+      }
+    }
+  }
+  if (!valid) return;
+  uint8_t* crow = codes + row * d + i1 + sub * C;
+#pragma unroll
+  for (int q = 0; q < C / 4; ++q) reinterpret_cast<uint32_t*>(crow)[q] = cw[q];
+  float* erow = err_out + row * B + sub * C;
+#pragma unroll
+  for (int q = 0; q < C / 4; ++q)
+    *reinterpret_cast<float4*>(erow + 4 * q) = make_float4(er[4 * q], er[4 * q + 1], er[4 * q + 2], er[4 * q + 3]);
 }
 
 // Whole quantization of 8 rows per CTA in one launch (layers whose U stays in L2): for every block,
@@ -448,9 +542,10 @@ template <int NS>
 gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, int gs, uint8_t* codes,
                        float* scales, int32_t* zeros, float* err, bool fma, int32_t* status, cudaStream_t s) {
   constexpr int B = 32 * NS;
-  const int smem = (B * B + B) * sizeof(float);
-  GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const int grid_rows = (int)((m + kRowsPerCta - 1) / kRowsPerCta);
+  constexpr int kLoopRows = 32;  // colloop_kernel: 4 warps of 8 rows
+  const int smem = (B * (B + 16) + B) * sizeof(float);
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<B / 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int grid_rows = (int)((m + kLoopRows - 1) / kLoopRows);
   CUtensorMap mErr, mU, mW;
   const bool tc = !fma && status != nullptr && tf32x3_map(&mErr, err, m, B, B, 128) &&
                   tf32x3_map(&mU, U, d, d, d, 32, true) && tf32x3_map(&mW, ww, m, d, d, 32);
@@ -464,7 +559,7 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
   g.status = status;
   const int tiles_m = (int)((m + 127) / 128);
   for (int i1 = 0; i1 < d; i1 += B) {
-    colloop_kernel<NS><<<grid_rows, 256, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
+    colloop_kernel<B / 4><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {
