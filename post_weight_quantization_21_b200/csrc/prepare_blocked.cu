@@ -104,12 +104,13 @@ __device__ void warp_factor_invert_128(const float* A, float* Li, int d, int piv
 // pass loop stays rolled: these products run once each per launch, so a compact body keeps the
 // kernel inside the instruction cache.  Ends with a barrier.  beta is 0 or 1.
 template <bool TB>
-__device__ void block_mm(float* out, const float* A, const float* B, int M, int N, int K, float alpha, float beta) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ void block_mm_w(float* out, const float* A, const float* B, int M, int N, int K, float alpha, float beta,
+                           int w0, int nw) {
+  const int warp = (threadIdx.x >> 5) - w0, lane = threadIdx.x & 31;
   const int mi = lane >> 2, ni = lane & 3;
   const int wn = N / 16, n_wt = (M / 16) * wn;
 #pragma unroll 1
-  for (int wt = warp; wt < n_wt; wt += 8) {
+  for (int wt = warp; wt < n_wt; wt += nw) {
     float r[2][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
@@ -152,8 +153,16 @@ __device__ void block_mm(float* out, const float* A, const float* B, int M, int 
         *e = (beta != 0.0f ? *e : 0.0f) + alpha * r[i][j];
       }
   }
+}
+
+template <bool TB>
+__device__ void block_mm(float* out, const float* A, const float* B, int M, int N, int K, float alpha, float beta) {
+  block_mm_w<TB>(out, A, B, M, N, K, alpha, beta, 0, 8);
   __syncthreads();
 }
+
+// barrier of warps 1-7 (the helpers of the diagonal-block factorisation)
+__device__ __forceinline__ void helpers_sync() { asm volatile("bar.sync 1, 224;" ::: "memory"); }
 
 // Factors the 128x128 diagonal block p and writes side[p] = L(p,p)^-1 (row-major, zeros above the
 // diagonal).  With `update` (p > 0) the block first receives its last update,
@@ -211,35 +220,45 @@ __device__ void factor_block(const float* P, int d, int p, bool update, float* s
   }
   __syncthreads();
   if (update) block_mm<true>(A, S, S, BB, BB, BB, -1.0f, 1.0f);  // A -= L(p,p-1) L(p,p-1)^T (S is free after)
+  // Four 32-wide steps.  Warp 0 factors diagonal block s (the chain); meanwhile warps 1-7 finish what
+  // step s-1 left that block s does not need: the panel solves of rows below s+1, the trailing
+  // update, and row band s-1 of the inverse.  Only the next row band's solve and the next diagonal
+  // block's update stay on the chain.  L blocks go to S (row band t, column band s), the inverse
+  // Y = L^-1 builds up in Li (zeros above the diagonal), and the band products' scratch Z uses the
+  // strictly upper part of A's first row band, which nothing else writes.
+  auto blk = [](float* M, int t, int c) { return M + t * kSub * LDS + c * kSub; };
+  float* Z = A + kSub;  // rows 0..31, columns 32..127 of A
+  constexpr int NSUB = BB / kSub;
 #pragma unroll 1
-  for (int s = 0; s < BB / kSub; ++s) {
-    float* Ass = A + s * kSub * LDS + s * kSub;
-    if (threadIdx.x < 32) warp_factor_invert_128(Ass, Li + s * kSub * LDS + s * kSub, d, p0 + s * kSub, status);
-    __syncthreads();
-    const int rest = BB - (s + 1) * kSub;
-    if (rest > 0) {
-      float* Ats = A + (s + 1) * kSub * LDS + s * kSub;
-      float* Sts = S + (s + 1) * kSub * LDS + s * kSub;
-      block_mm<true>(Sts, Ats, Li + s * kSub * LDS + s * kSub, rest, kSub, kSub, 1.0f, 0.0f);  // L(t, s), into S
-      for (int e = threadIdx.x; e < rest * kSub / 4; e += blockDim.x) {  // ... and back into A
-        const int r = e / (kSub / 4), c = (e % (kSub / 4)) * 4;
-        *reinterpret_cast<float4*>(Ats + r * LDS + c) = *reinterpret_cast<const float4*>(Sts + r * LDS + c);
+  for (int st = 0; st < NSUB; ++st) {
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+      warp_factor_invert_128(blk(A, st, st), blk(Li, st, st), d, p0 + st * kSub, status);
+    } else if (st >= 1) {
+      const int q = st - 1;  // the previous step
+      const int below = NSUB - 1 - st;  // row bands after st
+      if (below > 0)  // L(t, q) for t > st
+        block_mm_w<true>(blk(S, st + 1, q), blk(A, st + 1, q), blk(Li, q, q), below * kSub, kSub, kSub, 1.0f, 0.0f, 1, 7);
+      helpers_sync();
+      if (below > 0)  // A(t, c) -= L(t, q) L(c, q)^T for t > st, c >= st (upper tiles included, unused)
+        block_mm_w<true>(blk(A, st + 1, st), blk(S, st + 1, q), blk(S, st, q), below * kSub, (below + 1) * kSub, kSub,
+                         -1.0f, 1.0f, 1, 7);
+      if (q >= 1) {  // inverse row band q: Y(q, 0..q-1) = -Li(q,q) L(q, 0..q-1) Y(0..q-1, 0..q-1)
+        block_mm_w<false>(Z, blk(S, q, 0), Li, kSub, q * kSub, q * kSub, 1.0f, 0.0f, 1, 7);
+        helpers_sync();
+        block_mm_w<false>(blk(Li, q, 0), blk(Li, q, q), Z, kSub, q * kSub, kSub, -1.0f, 0.0f, 1, 7);
       }
-      __syncthreads();
-      float* Atr = A + (s + 1) * kSub * LDS + (s + 1) * kSub;
-      block_mm<true>(Atr, Sts, Sts, rest, rest, kSub, -1.0f, 1.0f);  // trailing part of the block
+    }
+    __syncthreads();
+    if (st + 1 < NSUB) {
+      // the chain: L(st+1, st), then the last update of diagonal block st+1
+      block_mm<true>(blk(S, st + 1, st), blk(A, st + 1, st), blk(Li, st, st), kSub, kSub, kSub, 1.0f, 0.0f);
+      block_mm<true>(blk(A, st + 1, st + 1), blk(S, st + 1, st), blk(S, st + 1, st), kSub, kSub, kSub, -1.0f, 1.0f);
     }
   }
-  // [[A,0],[C,B]]^-1 = [[A^-1, 0], [-B^-1 C A^-1, B^-1]], 32 -> 64 -> 128
-#pragma unroll 1
-  for (int h = kSub; h < BB; h *= 2) {
-#pragma unroll 1
-    for (int a0 = 0; a0 < BB; a0 += 2 * h) {
-      const int b0 = a0 + h;
-      block_mm<false>(S, A + b0 * LDS + a0, Li + a0 * LDS + a0, h, h, h, 1.0f, 0.0f);
-      block_mm<false>(Li + b0 * LDS + a0, Li + b0 * LDS + b0, S, h, h, h, -1.0f, 0.0f);
-    }
-  }
+  // inverse row band NSUB-1
+  block_mm<false>(Z, blk(S, NSUB - 1, 0), Li, kSub, (NSUB - 1) * kSub, (NSUB - 1) * kSub, 1.0f, 0.0f);
+  block_mm<false>(blk(Li, NSUB - 1, 0), blk(Li, NSUB - 1, NSUB - 1), Z, kSub, (NSUB - 1) * kSub, kSub, -1.0f, 0.0f);
   float4* out = reinterpret_cast<float4*>(side + (size_t)p * BB * BB);
   for (int e = threadIdx.x; e < BB * BB / 4; e += blockDim.x) {
     const int i = e / (BB / 4), c = (e % (BB / 4)) * 4;
