@@ -53,32 +53,28 @@ struct PrepArgs {
 };
 
 // ------------------------------------------------------------------ grid barrier (bounded)
-// Arrival counter and generation word sit in different 128-byte lines; waiters poll the generation
-// with acquire loads (no read-modify-write traffic on the line the arrivals update).
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
+// Grid barrier over a monotonically increasing arrival count (zeroed before the launch): barrier
+// number g is complete once the count reaches g * gridDim.x, so arriving is one atomic and waiting
+// is polling that word; no reset or separate release word is needed.  The wait is bounded.
 __device__ bool grid_barrier(const PrepArgs& a, unsigned& gen) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    const unsigned target = gen + 1;
+    const unsigned target = (gen + 1) * gridDim.x;
     unsigned* count = a.bar;
-    unsigned* generation = a.bar + 32;
     __threadfence();
-    const unsigned arrived = atomicAdd(count, 1u);
-    if (arrived == gridDim.x - 1) {
-      *(volatile unsigned*)count = 0u;
-      __threadfence();
-      atomicExch(generation, target);
-    } else {
+    const unsigned arrived = atomicAdd(count, 1u) + 1u;
+    if (arrived != target) {
       const long long t0 = clock64();
-      unsigned ns = 32;
-      while (ld_acquire(generation) != target) {
+      unsigned ns = 16;
+      while (ld_acquire(count) < target) {
         if (*(volatile int*)a.abort_flag) {
           ok = 0;
           break;
@@ -90,11 +86,11 @@ __device__ bool grid_barrier(const PrepArgs& a, unsigned& gen) {
           break;
         }
         __nanosleep(ns);
-        if (ns < 256) ns *= 2;
+        if (ns < 64) ns *= 2;
       }
     }
     __threadfence();
-    gen = target;
+    gen += 1;
     s_ok = ok;
   }
   __syncthreads();
@@ -268,7 +264,27 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(const PrepArgs a) {
     const int per_c = chunks > 0 ? chunks : 1;
     const int n_inv = (j >= 1) ? j * per_c : 0;
     const int n_items = n_panel + n_trail + n_inv;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    // Item assignment.  A panel item (~6 us: its 32x32 factorisation) or an inverse item (~5 us)
+    // gets a CTA of its own; the short trailing items share the remaining CTAs.  Handing a second
+    // item to a panel CTA would stretch the phase, and every CTA waits for the longest one.
+    const int G = gridDim.x;
+    const bool by_role = n_panel + n_inv < G;
+    for (int k = 0;; ++k) {
+      int it;
+      if (!by_role) {
+        it = blockIdx.x + k * G;
+        if (it >= n_items) break;
+      } else if ((int)blockIdx.x < n_panel) {
+        if (k > 0) break;
+        it = blockIdx.x;
+      } else if ((int)blockIdx.x < n_panel + n_inv) {
+        if (k > 0) break;
+        it = n_panel + n_trail + ((int)blockIdx.x - n_panel);
+      } else {
+        const int t = ((int)blockIdx.x - n_panel - n_inv) + k * (G - n_panel - n_inv);
+        if (t >= n_trail) break;
+        it = n_panel + t;
+      }
       float acc[2][4], acc2[2][4];
       if (it < n_panel) {
         // ------------------------------------------------ panel item
