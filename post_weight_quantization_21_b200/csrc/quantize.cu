@@ -171,25 +171,27 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
                : "memory");
 }
 
-// Column loop over block [i1, i1 + B) on the per-block launch path, 32 rows per CTA of 4 warps.
-// Four lanes (a quad) share a row: lane `sub` of the quad holds the C = B/4 consecutive columns
-// i1 + sub*C .. i1 + sub*C + C-1 in registers.  At block column i the owner lane (sub = i / C)
-// rounds its column, updates its own next column straight away (its chain stays in its registers
-// for C steps), and the error reaches the quad with one shuffle; each lane then applies it to its
-// columns after i.  The rounding runs once per warp instruction for 8 rows, so a row-step costs a
-// few warp instructions instead of a whole warp's.  The raw U block (B x B) sits in shared memory
-// with each row's four C-column chunks 16 bytes apart, so the quad's float4 reads of a row fall in
-// distinct bank groups; err * U[i, j] with err = delta / U_ii is the page's update.
-template <int C>
-__global__ void __launch_bounds__(128) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
+// Column loop over block [i1, i1 + B) on the per-block launch path, CTAs of 4 warps.  LPR lanes
+// share a row (32 / LPR rows per warp): lane `sub` of the row's group holds the C = B/LPR
+// consecutive columns i1 + sub*C .. i1 + sub*C + C-1 in registers.  At block column i the owner lane
+// (sub = i / C) rounds its column, updates its own next column straight away (its chain stays in its
+// registers for C steps), and the error reaches the group with one shuffle; each lane then applies
+// it to its columns after i.  The rounding runs once per warp instruction for 32 / LPR rows, so a
+// row-step costs a few warp instructions instead of a whole warp's; LPR = 8 gives layers with fewer
+// rows twice the warps (the step latency needs several warps per scheduler to hide).  The raw U
+// block (B x B) sits in shared memory with each row's C-column chunks padded apart so the group's
+// float4 reads of a row fall in distinct bank groups; err * U[i, j] with err = delta / U_ii is the
+// page's update.
+template <int C, int LPR>
+__global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
                                                       const float* __restrict__ U, int bits,
                                                       int group_size, uint8_t* __restrict__ codes,
                                                       float* __restrict__ scales,
                                                       int32_t* __restrict__ zeros,
                                                       float* __restrict__ err_out) {
-  constexpr int B = 4 * C;
-  constexpr int CS = C + 4;   // chunk stride
-  constexpr int RS = 4 * CS;  // row stride
+  constexpr int B = LPR * C;
+  constexpr int CS = ((C + 4) / 4) % 2 == 1 ? C + 4 : C + 8;  // chunk stride: an odd number of 16-byte granules
+  constexpr int RS = LPR * CS;                                  // row stride
   extern __shared__ __align__(16) float sm[];
   float* Ub = sm;             // U[i1 + r][i1 + q*C + t] at Ub[r*RS + q*CS + t]
   float* invd = sm + B * RS;  // 1 / U_ii
@@ -201,9 +203,9 @@ __global__ void __launch_bounds__(128) colloop_kernel(float* __restrict__ w, int
   if (threadIdx.x < B) invd[threadIdx.x] = 1.0f / U[(size_t)(i1 + threadIdx.x) * d + i1 + threadIdx.x];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane & 3;
-  const int qbase = lane & ~3;
-  const int64_t row = ((int64_t)blockIdx.x * (blockDim.x / 32) + warp) * 8 + (lane >> 2);
+  const int sub = lane & (LPR - 1);
+  const int qbase = lane & ~(LPR - 1);
+  const int64_t row = ((int64_t)blockIdx.x * (blockDim.x / 32) + warp) * (32 / LPR) + lane / LPR;
   const bool valid = row < m;  // lanes past the last row keep shuffling with zeros
   const int n_groups = group_size ? d / group_size : 1;
   float* wrow = w + (valid ? row : 0) * d;
@@ -227,12 +229,28 @@ __global__ void __launch_bounds__(128) colloop_kernel(float* __restrict__ w, int
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
+  // U row of the current step in registers, the next step's row loaded one step ahead (issue is in
+  // program order: loads made just before their FMAs would put the shared-memory latency on every step)
+  float4 un[C / 4];
+#pragma unroll
+  for (int q = 0; q < C / 4; ++q) un[q] = reinterpret_cast<const float4*>(Ub + sub * CS)[q];
+  float inv_next = invd[0];
 #pragma unroll 1
-  for (int o = 0; o < 4; ++o) {
+  for (int o = 0; o < LPR; ++o) {
     const bool owner = (sub == o);
 #pragma unroll
     for (int s = 0; s < C; ++s) {
       const int i = o * C + s;  // block column
+      float4 u[C / 4];
+#pragma unroll
+      for (int q = 0; q < C / 4; ++q) u[q] = un[q];
+      const float inv_i = inv_next;
+      if (i + 1 < B) {
+        const float* unext = Ub + (i + 1) * RS + sub * CS;
+#pragma unroll
+        for (int q = 0; q < C / 4; ++q) un[q] = reinterpret_cast<const float4*>(unext)[q];
+        inv_next = invd[i + 1];
+      }
       if (s == 0 && group_size != 0 && ((i1 + i) % group_size) == 0) {
         // grid of the group starting here, from the current values of its columns
         const int gend = i + group_size;  // block-local end (may pass the block)
@@ -246,15 +264,16 @@ __global__ void __launch_bounds__(128) colloop_kernel(float* __restrict__ w, int
           }
         }
         if (valid)
-          for (int c = i1 + B + sub; c < i1 + gend; c += 4) {  // group wider than the rest of the block
+          for (int c = i1 + B + sub; c < i1 + gend; c += LPR) {  // group wider than the rest of the block
             const float x = wrow[c];
             mn = fminf(mn, x);
             mx = fmaxf(mx, x);
           }
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+#pragma unroll
+        for (int x = 1; x < LPR; x <<= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, x));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+        }
         grid_from_range(mn, mx, maxq, scale, zero, rscale);
         if (sub == 0 && valid) {
           const int g = (i1 + i) / group_size;
@@ -266,25 +285,19 @@ __global__ void __launch_bounds__(128) colloop_kernel(float* __restrict__ w, int
       // code - zero, clamped to the grid; the quotient as an IEEE fp32 product with 1/scale
       const float qz = fminf(fmaxf(rintf(__fmul_rn(wi, rscale)), -zero), maxq - zero);
       const float delta = fmaf(-scale, qz, wi);  // w_i - dequantized value
-      const float err = delta * invd[i];
-      const float* urow = Ub + i * RS + sub * CS;
-      if (owner) {
-        cw[s >> 2] |= (uint32_t)(qz + zero) << (8 * (s & 3));
-        er[s] = err;
-        if (s + 1 < C) v[s + 1] = fmaf(-err, urow[s + 1], v[s + 1]);  // the owner's next column first
-      }
+      const float err = delta * inv_i;
+      // the owner keeps its code and error and updates its own next column straight away
+      // (selects rather than a branch: every lane runs the same instructions)
+      const float* ur = reinterpret_cast<const float*>(u);
+      cw[s >> 2] |= owner ? ((uint32_t)(qz + zero) << (8 * (s & 3))) : 0u;
+      er[s] = owner ? err : er[s];
+      if (s + 1 < C) v[s + 1] = owner ? fmaf(-err, ur[s + 1], v[s + 1]) : v[s + 1];
       const float e = __shfl_sync(0xffffffffu, err, qbase | o);
       // columns after i: every column of a lane past the owner, the owner's columns after s + 1
       const float f_near = (sub > o) ? e : 0.0f;
       const float f_far = (sub >= o) ? e : 0.0f;
 #pragma unroll
-      for (int q = 0; q < C / 4; ++q) {
-        const float4 u = reinterpret_cast<const float4*>(urow)[q];
-        v[4 * q + 0] = fmaf(4 * q + 0 <= s + 1 ? -f_near : -f_far, u.x, v[4 * q + 0]);
-        v[4 * q + 1] = fmaf(4 * q + 1 <= s + 1 ? -f_near : -f_far, u.y, v[4 * q + 1]);
-        v[4 * q + 2] = fmaf(4 * q + 2 <= s + 1 ? -f_near : -f_far, u.z, v[4 * q + 2]);
-        v[4 * q + 3] = fmaf(4 * q + 3 <= s + 1 ? -f_near : -f_far, u.w, v[4 * q + 3]);
-      }
+      for (int t = 0; t < C; ++t) v[t] = fmaf(t <= s + 1 ? -f_near : -f_far, ur[t], v[t]);
     }
   }
   if (!valid) return;
@@ -542,10 +555,17 @@ template <int NS>
 gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, int gs, uint8_t* codes,
                        float* scales, int32_t* zeros, float* err, bool fma, int32_t* status, cudaStream_t s) {
   constexpr int B = 32 * NS;
-  constexpr int kLoopRows = 32;  // colloop_kernel: 4 warps of 8 rows
-  const int smem = (B * (B + 16) + B) * sizeof(float);
-  GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<B / 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const int grid_rows = (int)((m + kLoopRows - 1) / kLoopRows);
+  // lanes per row of the column loop: 8 while that still leaves about 7 warps per SM, else 4
+  const bool lpr8 = m <= 6144;
+  constexpr int C4 = B / 4, C8 = B / 8;
+  constexpr int CS4 = ((C4 + 4) / 4) % 2 == 1 ? C4 + 4 : C4 + 8, CS8 = ((C8 + 4) / 4) % 2 == 1 ? C8 + 4 : C8 + 8;
+  const int loop_rows = lpr8 ? 16 : 32;  // 4 warps of 32 / LPR rows
+  const int smem = (B * (lpr8 ? 8 * CS8 : 4 * CS4) + B) * (int)sizeof(float);
+  if (lpr8)
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<C8, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  else
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<C4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int grid_rows = (int)((m + loop_rows - 1) / loop_rows);
   CUtensorMap mErr, mU, mW;
   const bool tc = !fma && status != nullptr && tf32x3_map(&mErr, err, m, B, B, 128) &&
                   tf32x3_map(&mU, U, d, d, d, 32, true) && tf32x3_map(&mW, ww, m, d, d, 32);
@@ -559,7 +579,10 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
   g.status = status;
   const int tiles_m = (int)((m + 127) / 128);
   for (int i1 = 0; i1 < d; i1 += B) {
-    colloop_kernel<B / 4><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
+    if (lpr8)
+      colloop_kernel<C8, 8><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
+    else
+      colloop_kernel<C4, 4><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {

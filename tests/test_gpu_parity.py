@@ -120,6 +120,7 @@ PER_BLOCK_CASES = [
     (2100, 256, 4, 0, 128),
     (2500, 512, 3, 128, 128),
     (2049, 256, 4, 0, 32),
+    (6200, 256, 3, 0, 128),    # past 6144 rows: four lanes per row in the column loop
     (40, 4224, 3, 128, 128),
     (24, 4352, 4, 0, 64),
 ]
