@@ -51,6 +51,15 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return
 // scale = (hi - lo) / maxq in IEEE fp32, rscale = IEEE fp32 reciprocal of scale, and
 // zero = rint(-lo * rscale).  Quotients that decide an integer are always formed as x * rscale
 // (IEEE fp32 product, not contracted into an FMA).
+// Round to the nearest integer, ties to even, with two fp32 adds on the FMA pipe: adding 1.5 * 2^23
+// moves |x| < 2^22 into [2^23, 2^24), where the spacing of floats is 1, so the addition itself rounds.
+// Equal to rintf(x) for |x| < 2^22; larger magnitudes come out at least 2^22 - 1 in magnitude, beyond
+// any b-bit grid, so a following clamp gives the same result as with rintf.
+__device__ __forceinline__ float round_even(float x) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  return __fsub_rn(__fadd_rn(x, kShift), kShift);
+}
+
 __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, float& scale,
                                                 float& zero, float& rscale) {
   float lo = fminf(mn, 0.0f);

@@ -53,8 +53,9 @@ __global__ void __launch_bounds__(256) convert_rowgrid_kernel(const T* __restric
 //
 // Step i (owner lane L = i / NS, slot s = i % NS): every lane rounds its own v[s] (only the owner's
 // result is kept), the owner's error is broadcast, and every lane applies err * U[i, j] to its
-// columns.  The owner updates its next column from its own error before the broadcast lands, so the
-// dependency chain leaves the lane only once every NS steps.
+// columns after i.  The owner updates its next column from its own error before the broadcast lands,
+// so the dependency chain leaves the lane only once every NS steps; the U row of the next step is
+// read one step ahead.
 template <int NS>
 __device__ __forceinline__ void column_loop(float (&v)[NS], const float* __restrict__ Us,
                                             const float* __restrict__ invd, int i1, int group_size,
@@ -64,11 +65,35 @@ __device__ __forceinline__ void column_loop(float (&v)[NS], const float* __restr
                                             uint32_t (&code_reg)[NS], float (&err_reg)[NS]) {
   constexpr int B = 32 * NS;
   const int lane = threadIdx.x & 31;
+  // this lane's NS entries of the current U row, the next row loaded one step ahead
+  // one vector load per lane (NS consecutive floats, 4 * NS-byte aligned)
+  auto load_row = [&](float (&dst)[NS], const float* src) {
+    if constexpr (NS == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src);
+      dst[0] = x.x, dst[1] = x.y, dst[2] = x.z, dst[3] = x.w;
+    } else if constexpr (NS == 2) {
+      const float2 x = *reinterpret_cast<const float2*>(src);
+      dst[0] = x.x, dst[1] = x.y;
+    } else {
+      dst[0] = src[0];
+    }
+  };
+  float un[NS];
+  load_row(un, Us + lane * NS);
+  float inv_next = invd[0];
 #pragma unroll 1
   for (int L = 0; L < 32; ++L) {
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
       const int i = L * NS + s;
+      float u[NS];
+#pragma unroll
+      for (int t = 0; t < NS; ++t) u[t] = un[t];
+      const float inv_i = inv_next;
+      if (i + 1 < B) {
+        load_row(un, Us + (i + 1) * B + lane * NS);
+        inv_next = invd[i + 1];
+      }
       if (group_size != 0 && s == 0 && ((i1 + i) % group_size) == 0) {
         // grid of the group starting here, from the current values of its columns
         const int c_end = i + group_size;  // block-local end (may pass the block)
@@ -98,25 +123,20 @@ __device__ __forceinline__ void column_loop(float (&v)[NS], const float* __restr
       const bool owner = (lane == L);
       const float wi = owner ? v[s] : 0.0f;  // only the owner's value matters
       // code - zero, clamped to the grid; the quotient as an IEEE fp32 product with 1/scale
-      const float qz = fminf(fmaxf(rintf(__fmul_rn(wi, rscale)), -zero), maxq - zero);
+      const float qz = fminf(fmaxf(round_even(__fmul_rn(wi, rscale)), -zero), maxq - zero);
       const float delta = fmaf(-scale, qz, wi);  // w_i - dequantized value
-      const float err = delta * invd[i];
-      if (owner) {
-        code_reg[s] = (uint32_t)(qz + zero);
-        err_reg[s] = err;
-      }
+      const float err = delta * inv_i;
+      // selects rather than branches: every lane runs the same instructions
+      code_reg[s] = owner ? (uint32_t)(qz + zero) : code_reg[s];
+      err_reg[s] = owner ? err : err_reg[s];
       // Us rows are pre-divided by U_ii: err * U[i][j] = delta * Us[i][j]
-      const float* urow = Us + i * B + lane * NS;
-      if (s + 1 < NS && owner) v[s + 1] = fmaf(-delta, urow[s + 1], v[s + 1]);  // owner's next column first
+      if (s + 1 < NS) v[s + 1] = owner ? fmaf(-delta, u[s + 1], v[s + 1]) : v[s + 1];  // owner's next column first
       const float e = __shfl_sync(0xffffffffu, delta, L);
+      // columns after i: every column of a lane past the owner, the owner's columns after s + 1
+      const float f_near = (lane > L) ? e : 0.0f;
+      const float f_far = (lane >= L) ? e : 0.0f;
 #pragma unroll
-      for (int t = 0; t < NS; ++t) {
-        if (t == s + 1) {
-          if (!owner) v[t] = fmaf(-e, urow[t], v[t]);
-        } else {
-          v[t] = fmaf(-e, urow[t], v[t]);
-        }
-      }
+      for (int t = 0; t < NS; ++t) v[t] = fmaf(t <= s + 1 ? -f_near : -f_far, u[t], v[t]);
     }
   }
 }
@@ -283,7 +303,7 @@ __global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, 
       }
       const float wi = v[s];  // the owner's column (other lanes compute and discard)
       // code - zero, clamped to the grid; the quotient as an IEEE fp32 product with 1/scale
-      const float qz = fminf(fmaxf(rintf(__fmul_rn(wi, rscale)), -zero), maxq - zero);
+      const float qz = fminf(fmaxf(round_even(__fmul_rn(wi, rscale)), -zero), maxq - zero);
       const float delta = fmaf(-scale, qz, wi);  // w_i - dequantized value
       const float err = delta * inv_i;
       // the owner keeps its code and error and updates its own next column straight away
