@@ -332,8 +332,9 @@ __global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, 
 
 // Whole quantization of 8 rows per CTA in one launch (layers whose U stays in L2): for every block,
 // the column loop (one warp per row, U corner in shared memory), then the lazy update of the CTA's
-// rows, W[rows, i2:] -= Err[rows, :] U[i1:i2, i2:], with U streamed through shared memory in
-// 128-column chunks.  Rows are independent given U, so CTAs never wait on one another.
+// rows, W[rows, i2:] -= Err[rows, :] U[i1:i2, i2:], with U streamed through two shared-memory
+// buffers of 128 columns by cp.async (the next chunk lands while the current one is used).  Rows are
+// independent given U, so CTAs never wait on one another.
 template <typename T, int NS>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ W, int64_t m, int d,
                                                             const float* __restrict__ U, int bits,
@@ -344,9 +345,10 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
   constexpr int B = 32 * NS;
   constexpr int CW = 128;  // lazy-update chunk width (columns)
   extern __shared__ __align__(16) float sm[];
-  float* Us = sm;                // [B][B] corner of U, then [B][CW] chunks of the U panel
+  float* Us = sm;                // [B][B] corner of U, then [B][CW] chunks of the U panel (buffer 0)
   float* invd = sm + B * CW;     // [B]
   float* errs = invd + B;        // [8][B]
+  float* Us2 = errs + kRowsPerCta * B;  // [B][CW] chunk buffer 1
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + warp;
   const bool valid = row < m;
@@ -397,40 +399,37 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
         errs[warp * B + lane * NS + s] = err_reg[s];
       }
     }
-    // lazy update of this CTA's rows over the columns after the block; the next chunk of the U
-    // panel is loaded into registers while the current one is used from shared memory
-    constexpr int PER = B * CW / 4 / 256;  // float4 of a chunk per thread
-    float4 uv[PER];
-    auto fetch_chunk = [&](int c0) {
-#pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        const int e = threadIdx.x + 256 * k;
-        const int r = e / (CW / 4), c = (e % (CW / 4)) * 4;
-        uv[k] = (c0 + c < d) ? *reinterpret_cast<const float4*>(U + (size_t)(i1 + r) * d + c0 + c)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    // lazy update of this CTA's rows over the columns after the block, chunk by chunk; columns past
+    // d are not copied (no lane reads them)
+    const int n_chunks = (d - (i1 + B) + CW - 1) / CW;
+    auto issue_chunk = [&](int c, float* dst) {
+      const int c0 = i1 + B + c * CW;
+      for (int e = threadIdx.x; e < B * CW / 4; e += blockDim.x) {
+        const int r = e / (CW / 4), cc = (e % (CW / 4)) * 4;
+        if (c0 + cc < d) cp_async16(dst + r * CW + cc, U + (size_t)(i1 + r) * d + c0 + cc);
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    if (i1 + B < d) fetch_chunk(i1 + B);
-    for (int c0 = i1 + B; c0 < d; c0 += CW) {
-      const bool mine = valid && c0 + 4 * lane < d;
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (mine) o = *reinterpret_cast<const float4*>(wr + c0 + 4 * lane);
-      __syncthreads();
-#pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        const int e = threadIdx.x + 256 * k;
-        const int r = e / (CW / 4), c = (e % (CW / 4)) * 4;
-        *reinterpret_cast<float4*>(Us + r * CW + c) = uv[k];
+    __syncthreads();  // the column loop is done with the U corner in buffer 0
+    if (n_chunks > 0) issue_chunk(0, Us);
+    for (int c = 0; c < n_chunks; ++c) {
+      float* cur = (c & 1) ? Us2 : Us;
+      if (c + 1 < n_chunks) {
+        issue_chunk(c + 1, (c & 1) ? Us : Us2);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
       }
-      __syncthreads();
-      if (c0 + CW < d) fetch_chunk(c0 + CW);
-      if (mine) {
+      __syncthreads();  // chunk c has landed for every thread
+      const int c0 = i1 + B + c * CW;
+      if (valid && c0 + 4 * lane < d) {
+        float4 o = *reinterpret_cast<const float4*>(wr + c0 + 4 * lane);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         const float* er = errs + warp * B;
 #pragma unroll 8
         for (int k = 0; k < B; ++k) {
           const float e = er[k];
-          const float4 u = *reinterpret_cast<const float4*>(Us + k * CW + 4 * lane);
+          const float4 u = *reinterpret_cast<const float4*>(cur + k * CW + 4 * lane);
           acc.x = fmaf(e, u.x, acc.x);
           acc.y = fmaf(e, u.y, acc.y);
           acc.z = fmaf(e, u.z, acc.z);
@@ -442,6 +441,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
         o.w -= acc.w;
         *reinterpret_cast<float4*>(wr + c0 + 4 * lane) = o;
       }
+      __syncthreads();  // every thread is done with `cur` before chunk c + 2 is copied into it
     }
   }
 }
@@ -627,7 +627,7 @@ template <typename T, int NS>
 gptq_status launch_rows(const void* W, int64_t m, int d, const float* U, int bits, int gs, float* ww, uint8_t* codes,
                         float* scales, int32_t* zeros, cudaStream_t s) {
   constexpr int B = 32 * NS;
-  const int smem = (B * 128 + B + kRowsPerCta * B) * sizeof(float);
+  const int smem = (2 * B * 128 + B + kRowsPerCta * B) * sizeof(float);
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(quantize_rows_kernel<T, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid = (int)((m + kRowsPerCta - 1) / kRowsPerCta);
   quantize_rows_kernel<T, NS><<<grid, 256, smem, s>>>(static_cast<const T*>(W), m, d, U, bits, gs, ww, codes, scales,
