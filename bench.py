@@ -47,6 +47,24 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def slowest_rank_ms(ms: float, device) -> float:
+    """The largest of the ranks' device-timed values (a multi-GPU time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def layer_for_rank(L, rank: int):
+    """Rank r quantizes its own layer of the same shape (inputs seeded seed + r): weak scaling, no
+    data-path collective."""
+    import dataclasses
+    return dataclasses.replace(L, seed=L.seed + rank)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -197,6 +215,7 @@ def main():
     import post_weight_quantization_21_b200 as g
 
     rank, world, local = dist_env()
+    L = layer_for_rank(L, rank)
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
@@ -253,10 +272,7 @@ def main():
 
     total_ms = start.elapsed_time(end)
     phase_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = slowest_rank_ms(total_ms, dev)
     ms_per_step = total_ms / args.steps
     value = world * L.m * L.d / (ms_per_step * 1e-3)
 
@@ -280,10 +296,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = slowest_rank_ms(e2e_ms, dev)
     h2d = W_h.numel() * W_h.element_size() + X_h.numel() * X_h.element_size()
     d2h = sum(t.numel() * t.element_size() for t in (out_p, out_s, out_z))
 
