@@ -10,15 +10,19 @@
 //   factor(0)
 //   for each panel p:
 //     trsm(p)           L(r, p) = P(r, p) L(p,p)^-T for every row block r > p
-//     syrk(p)           P(r, c) -= L(r, p) L(c, p)^T for p < c <= r, except the block (p+1, p+1)
-//     factor(p+1)       one CTA: P(p+1,p+1) - L(p+1,p) L(p+1,p)^T, factored in four 32-wide steps
-//                       (each a one-warp factorisation) and inverted -> side[p+1] = L(p+1,p+1)^-1
+//     syrk(p)           P(r, c) -= L(r, p) L(c, p)^T for p < c <= r
+//     factor(p+1)       one CTA: the diagonal block (p+1, p+1) factored in four 32-wide steps (each a
+//                       one-warp factorisation, the rest overlapped by the other warps) and inverted
+//                       -> side[p+1] = L(p+1,p+1)^-1
 //   leaf_copy           diagonal blocks of P <- side
 //   for g = 1, 2, 4, ...: T = C A^-1, Y21 = -B^-1 T for [[A,0],[C,B]] pairs of g blocks
 //   rotate              U = J Y J
-// factor(p+1) depends only on trsm(p), so it runs on a second stream alongside syrk(p) (look-ahead):
-// the serial chain per panel is trsm + max(syrk, factor) instead of their sum.  The block products
-// run on one 128x128x128 fp32 tile kernel (8x8 outputs per thread).
+// factor(p+1) depends only on trsm(p) and the update of block (p+1, p+1), so that tile and the
+// factorisation run on a second stream alongside the rest of syrk(p) (look-ahead): the serial chain
+// per panel is trsm + max(syrk, diagonal tile + factor) instead of their sum.  The block products
+// run on the tensor cores as 3xTF32 (gemm_tf32x3.cu) when rows are 16-byte aligned (d % 4 == 0),
+// else on an fp32 FMA tile kernel below (128x128x128 tiles, 8x8 outputs per thread), where the
+// factorisation does the diagonal block's last update itself.
 #include <math.h>
 
 #include <mutex>

@@ -3,11 +3,16 @@
 // GPTQ's column loop (FDE Interviews breakdown of GPTQ, figure "THE IDEA, VISUALLY"):
 //   1. round column i to the b-bit grid;  2. err = (w_i - q_i) / U_ii;
 //   3. W[:, i+1:] -= err * U[i, i+1:];   4. apply in blocks of 128 columns.
-// Rows are independent once U is known (section 01: one column order shared by every row), so a
-// warp owns a row: lane l holds columns l, l+32, l+64, l+96 of the current block in registers and
-// the block's 128x128 corner of U sits in shared memory.  Each step broadcasts w_i with one
-// shuffle, rounds it, and updates the four register columns; the block never leaves the SM.
-// Step 4 is a separate tiled fp32 GEMM per block: W[:, i2:] -= Err[:, i1:i2] U[i1:i2, i2:].
+// Rows are independent once U is known (section 01: one column order shared by every row), so rows
+// are spread over lanes and the block's corner of U sits in shared memory; the block never leaves
+// the SM.  Two forms:
+//   - quantize_rows_kernel (layers whose U stays in L2, few rows): one warp per row, lane l holding
+//     NS consecutive columns of the block; after each block the CTA applies step 4 to its own rows,
+//     streaming U through shared memory.  One launch per layer.
+//   - colloop_kernel + a per-block lazy update (other layers): 4 or 8 lanes per row, so one warp
+//     instruction advances several rows; step 4 for all rows is a tensor-core 3xTF32 product
+//     W[:, i2:] -= Err[:, i1:i2] U[i1:i2, i2:] (gemm_tf32x3.cu), or lazy_gemm_kernel on the fp32 FMA
+//     units with GPTQ_FLAG_FP32_FMA.
 #include "common.cuh"
 #include "kernels.h"
 
