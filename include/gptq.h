@@ -106,8 +106,14 @@ GPTQ_API size_t gptq_hessian_workspace_size(int64_t n_tokens, int64_t d, int32_t
  *   U          [d, d] fp32 output: upper triangle = the factor, strict lower triangle = 0.
  *              Also used as scratch during the call; must not alias H.
  *   dev_status int32[2]: cleared at the start of the call; {GPTQ_ERR_NOT_PD, pivot column} if the
- *              dampened matrix is not positive definite (U is then unspecified).
+ *              dampened matrix is not positive definite (U is then unspecified); GPTQ_ERR_TIMEOUT
+ *              if a bounded device wait gave up.
  *   workspace  >= gptq_prepare_workspace_size(d) bytes, 256-byte aligned.
+ *   d <= 1024 runs as one cooperative launch.  Larger orders run a blocked factorisation whose block
+ *   products use the tensor cores as 3xTF32 when d % 4 == 0 (fp32 FMA tiles otherwise); their next
+ *   diagonal block is factored on a second stream that the library creates once per device (with
+ *   two events) and joins back into `stream` before the call's last launch, so the whole call is
+ *   ordered on `stream` for the caller.
  * ------------------------------------------------------------------------------------------ */
 GPTQ_API gptq_status gptq_prepare_uinv(const float* H, int64_t d, float damp, float* U, int32_t* dev_status,
                               void* workspace, size_t workspace_bytes, void* stream);
@@ -128,6 +134,7 @@ GPTQ_API size_t gptq_prepare_workspace_size(int64_t d);
  *   with that device current); make that first call before any stream capture.
  *   All calls share the one array and it keeps the last call's contents (each call clears the parts
  *   that must start at zero).  Calls that overlap on the GPU, on any streams, race on it: order them.
+ *   It creates no CUDA objects: above d = 1024 every launch goes to `stream` (no look-ahead stream).
  *   No memory is allocated or freed.
  * ------------------------------------------------------------------------------------------ */
 #define GPTQ_PREPARE_STATIC_MAX_D 8192
