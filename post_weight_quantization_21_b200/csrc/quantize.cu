@@ -592,7 +592,9 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<C4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid_rows = (int)((m + loop_rows - 1) / loop_rows);
   CUtensorMap mErr, mU, mW;
-  const bool tc = !fma && status != nullptr && tf32x3_map(&mErr, err, m, B, B, 128) &&
+  // the tensor-core update numbers its 128x128 tiles with 32-bit ints
+  const bool tiles_fit = ((m + 127) / 128) * (int64_t)((d + 127) / 128) <= 0x7fffffff;
+  const bool tc = !fma && status != nullptr && tiles_fit && tf32x3_map(&mErr, err, m, B, B, 128) &&
                   tf32x3_map(&mU, U, d, d, d, 32, true) && tf32x3_map(&mW, ww, m, d, d, 32);
   Tf32x3Args g{};
   g.kind = kGemmLazy;
