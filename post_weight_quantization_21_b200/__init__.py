@@ -210,6 +210,9 @@ class LayerSolver:
     inputs in, runs, and copies the packed codes, scales and zeros back out.
     """
 
+    HOST_CHUNK_TOKENS = 16384  # tokens of X per host -> device copy in run_host (a multiple of 64)
+
+
     def __init__(self, m: int, d: int, n_tokens: int, bits: int, group_size: int = 0, block_size: int = 128,
                  damp: float = 0.01, x_dtype=torch.bfloat16, w_dtype=torch.float16, device="cuda", flags: int = 0):
         self.m, self.d, self.n_tokens, self.flags = m, d, n_tokens, flags
@@ -225,19 +228,24 @@ class LayerSolver:
         self.scales = torch.empty(m, n_groups, dtype=torch.float32, device=dev)
         self.zeros = torch.empty(m, n_groups, dtype=torch.int32, device=dev)
         self.packed = torch.empty(m, d * bits // 32, dtype=torch.int32, device=dev)
-        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
-        ws = max(gptq_hessian_workspace_size(n_tokens, d, x_dtype), gptq_prepare_workspace_size(d),
-                 gptq_quantize_workspace_size(m, d, bits, group_size, block_size), 256)
+        # one device status word per call (prepare and quantize clear theirs when they start)
+        self.status = torch.zeros(3, 2, dtype=torch.int32, device=dev)  # rows: hessian, prepare, quantize
+        self.host_chunk = min(n_tokens, self.HOST_CHUNK_TOKENS)
+        ws = max(gptq_hessian_workspace_size(n_tokens, d, x_dtype),
+                 gptq_hessian_workspace_size(self.host_chunk, d, x_dtype) if self.host_chunk else 0,
+                 gptq_prepare_workspace_size(d), gptq_quantize_workspace_size(m, d, bits, group_size, block_size),
+                 256)
         self.workspace = torch.empty(ws, dtype=u8, device=dev)
+        self._copy_stream = None
 
     def hessian(self, stream=None):
-        gptq_hessian_accumulate(self.X, self.H, self.status, self.workspace, 2.0, False, stream)
+        gptq_hessian_accumulate(self.X, self.H, self.status[0], self.workspace, 2.0, False, stream)
 
     def prepare(self, stream=None):
-        gptq_prepare_uinv(self.H, self.U, self.status, self.workspace, self.damp, stream)
+        gptq_prepare_uinv(self.H, self.U, self.status[1], self.workspace, self.damp, stream)
 
     def quantize(self, stream=None):
-        gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.status, self.workspace,
+        gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.status[2], self.workspace,
                             self.bits, self.group_size, self.block_size, self.flags, stream)
 
     def pack(self, stream=None):
@@ -250,16 +258,45 @@ class LayerSolver:
         self.pack(stream)
 
     def check_status(self, stream=None):
-        code, detail = gptq_read_status(self.status, stream)
-        if code != GPTQ_OK:
-            raise GPTQError(code, "device status", detail)
+        """Raises GPTQError with the first failure any of the calls recorded on the device."""
+        for word in self.status:
+            code, detail = gptq_read_status(word, stream)
+            if code != GPTQ_OK:
+                raise GPTQError(code, "device status", detail)
 
     def run_host(self, W_host: torch.Tensor, X_host: torch.Tensor, out_packed: torch.Tensor,
                  out_scales: torch.Tensor, out_zeros: torch.Tensor, stream=None):
-        """Host -> device copies of W and X, the four calls, device -> host copies of the results."""
-        self.X.copy_(X_host, non_blocking=True)
-        self.W.copy_(W_host, non_blocking=True)
-        self.run(stream)
-        out_packed.copy_(self.packed, non_blocking=True)
-        out_scales.copy_(self.scales, non_blocking=True)
-        out_zeros.copy_(self.zeros, non_blocking=True)
+        """Host -> device copies of W and X, the four calls, device -> host copies of the results.
+
+        X crosses in chunks of HOST_CHUNK_TOKENS tokens on a copy stream, and the Hessian of each chunk
+        accumulates (gptq_hessian_accumulate with accumulate = 1) as soon as the chunk has landed, so
+        the copy of chunk c + 1 overlaps the product of chunk c.  W crosses first.  Inputs should be
+        pinned for the copies to be asynchronous.
+        """
+        s = stream if stream is not None else torch.cuda.current_stream(self.X.device)
+        if self._copy_stream is None:
+            self._copy_stream = torch.cuda.Stream(device=self.X.device)
+        copy = self._copy_stream
+        copy.wait_stream(s)  # the device buffers are free once the caller's earlier work is done
+        step = max(self.host_chunk, 1)
+        landed = []
+        with torch.cuda.stream(copy):
+            self.W.copy_(W_host, non_blocking=True)
+            for t0 in range(0, self.n_tokens, step):
+                self.X[t0:t0 + step].copy_(X_host[t0:t0 + step], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy)
+                landed.append(ev)
+        if not landed:  # no tokens: H = 0
+            s.wait_stream(copy)
+            gptq_hessian_accumulate(self.X, self.H, self.status[0], self.workspace, 2.0, False, s)
+        for c, t0 in enumerate(range(0, self.n_tokens, step)):
+            s.wait_event(landed[c])
+            gptq_hessian_accumulate(self.X[t0:t0 + step], self.H, self.status[0], self.workspace, 2.0, c > 0, s)
+        self.prepare(s)
+        self.quantize(s)
+        self.pack(s)
+        with torch.cuda.stream(s):
+            out_packed.copy_(self.packed, non_blocking=True)
+            out_scales.copy_(self.scales, non_blocking=True)
+            out_zeros.copy_(self.zeros, non_blocking=True)

@@ -208,3 +208,28 @@ def test_end_to_end_reduced_llama_q_layer():
     import dataclasses
     L = dataclasses.replace(L, m=512, d=1024, n_tokens=16 * 2048)
     _layer_end_to_end(L)
+
+
+def test_run_host_streams_x_in_chunks():
+    """LayerSolver.run_host: X crosses in HOST_CHUNK_TOKENS chunks whose Hessians accumulate as they land
+    (a ragged last chunk of 40 tokens takes the fp32 Hessian path); results match the oracle."""
+    m, d, bits, gs = 256, 512, 4, 128
+    n = 2 * g.LayerSolver.HOST_CHUNK_TOKENS + 40
+    gen = torch.Generator().manual_seed(9)
+    X = (torch.randn(n, d, generator=gen) @ (torch.randn(d, d, generator=gen) / d ** 0.5)).to(torch.bfloat16)
+    W = (torch.randn(m, d, generator=gen) * 0.02).half()
+    s = g.LayerSolver(m, d, n, bits, gs, 128, 0.01, X.dtype, W.dtype, device=S.dev())
+    n_groups = d // gs
+    out_p = torch.empty(m, d * bits // 32, dtype=torch.int32).pin_memory()
+    out_s = torch.empty(m, n_groups, dtype=torch.float32).pin_memory()
+    out_z = torch.empty(m, n_groups, dtype=torch.int32).pin_memory()
+    s.run_host(W.pin_memory(), X.pin_memory(), out_p, out_s, out_z)
+    torch.cuda.synchronize()
+    s.check_status()
+    H = oracle.hessian(X.double().numpy())
+    assert S.upper_rel_fro(s.H.double().cpu().numpy(), H) <= S.H_REL_FRO
+    U = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01))
+    ref = oracle.gptq_quantize(W.double().numpy(), U, bits, gs, 128)
+    codes = oracle.unpack_codes(out_p.numpy(), bits, d).astype(np.int64)
+    S.compare_quantization((codes, out_s.numpy(), out_z.numpy().astype(np.int64)), ref, gs, W.double().numpy(), H,
+                           label="run_host")
