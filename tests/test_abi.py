@@ -100,3 +100,13 @@ def test_tensor_core_phase_mask_without_a_device():
                                      flags=g.GPTQ_FLAG_FP32_FMA) == g.GPTQ_TC_HESSIAN | g.GPTQ_TC_PREPARE
     assert g.gptq_tensor_core_phases(64, 4224, 256, torch.float32, 4) == g.GPTQ_TC_PREPARE | g.GPTQ_TC_LAZY
     assert g.gptq_tensor_core_phases(64, 100, 256, torch.float32, 4) == -1   # block does not divide d
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No fallback: without libgptq.so every call raises instead of computing anything elsewhere."""
+    monkeypatch.setattr(g, "LIB_PATH", str(tmp_path / "libgptq.so"))
+    monkeypatch.setattr(g, "_lib", None)
+    with pytest.raises(ImportError):
+        g.lib()
+    with pytest.raises(ImportError):
+        g.gptq_prepare_workspace_size(128)
