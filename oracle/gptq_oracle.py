@@ -17,15 +17,14 @@ Sources (web pages about GPTQ, Frantar, Ashkboos, Hoefler, Alistarh, ICLR 2023):
 [CSDN] "GPTQ量化参数搜索工具", agent.csdn.net: 关键参数说明 table (bits, group_size, zero point).
 
 Precision.  Every floating-point step is fp64, except the two places where a floating-point value
-decides an integer (the zero point and the code of each weight).  There both the oracle and the CUDA
-path take the decision in fp32 (the kernels' precision) with the same operation sequence: the
-quotient x / scale is formed as the IEEE round-to-nearest fp32 product of x and the IEEE fp32
-reciprocal of the scale, then rounded half-to-even, so equal operands give equal integers.
+decides an integer (the zero point and the code of each weight).  There the decision is taken in
+fp32, the precision of the CUDA kernels: the quotient x / scale is the IEEE round-to-nearest fp32
+quotient of the fp32 operands, then rounded half-to-even.
 
 Readings of the pages (they are silent or garbled here; the plainest reading is used):
 * Grid: asymmetric min/max uniform grid on {0..2^b-1}; the range is widened to contain 0; an all-zero
-  range becomes [-1, 1]; zero = rint(-xmin/scale); q = clamp(rint(x/scale) + zero, 0, maxq), with the
-  quotients formed as x * (1/scale) in fp32 (see Precision).
+  range becomes [-1, 1]; zero = rint(-xmin/scale); q = clamp(rint(x/scale) + zero, 0, maxq), the
+  quotients taken in fp32 (see Precision).
 * Per-row grids come from the original row before the column loop; per-group grids come from the
   current (already compensated) values of the group's columns when the loop reaches the group.
 * The column loop quantizes the current, compensated value of each column ([FDE] figure, step 1),
@@ -139,19 +138,14 @@ def grid_params(xmin, xmax, bits: int):
     lo = np.where(flat, np.float32(-1.0), lo)
     hi = np.where(flat, np.float32(1.0), hi)
     scale = ((hi - lo) / maxq).astype(np.float32)
-    zero = np.rint((-lo) * _recip32(scale)).astype(np.float32)
+    zero = np.rint(((-lo) / scale).astype(np.float32))
     return scale, zero.astype(np.int64)
 
 
-def _recip32(scale):
-    """IEEE fp32 reciprocal of the (fp32) scale."""
-    return (np.float32(1.0) / np.asarray(scale, dtype=np.float32)).astype(np.float32)
-
-
 def quantize_codes(x, scale, zero, bits: int) -> np.ndarray:
-    """q = clamp(rint(x / scale) + zero, 0, 2^b - 1), the quotient formed in fp32 as x * (1/scale)."""
+    """q = clamp(rint(x / scale) + zero, 0, 2^b - 1), the quotient an IEEE fp32 division."""
     x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
-    r = np.rint((x32 * _recip32(scale)).astype(np.float32)).astype(np.int64)
+    r = np.rint((x32 / np.asarray(scale, dtype=np.float32)).astype(np.float32)).astype(np.int64)
     return np.clip(r + np.asarray(zero, dtype=np.int64), 0, 2 ** bits - 1)
 
 

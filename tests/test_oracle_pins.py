@@ -127,6 +127,37 @@ def test_worked_example_d3(golden_dir):
                                   np.array(g["rtn_codes"], dtype=int))
 
 
+def _group_golden(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "worked_example_group.txt"))
+    Hd = np.array(g["hd"], dtype=float).reshape(4, 4)
+    w = np.array(g["w"], dtype=float)[None, :]
+    return g, Hd, w, int(g["bits"][0]), int(g["group_size"][0])
+
+
+def _check_group_golden(g, Hd, w, bits, gs, block_size):
+    """True when the oracle reproduces every hand-worked value of the group example."""
+    U = O.inverse_upper_cholesky(Hd)
+    r = O.gptq_quantize(w, U, bits, gs, block_size)
+    comp = r["Wq"][0] + r["Err"][0] * np.diag(U)
+    return (np.array_equal(r["codes"][0], np.array(g["codes"], dtype=int))
+            and np.allclose(r["scales"][0], np.array(g["scales"], dtype=float), rtol=1e-6, atol=0)
+            and np.array_equal(r["zeros"][0], np.array(g["zeros"], dtype=int))
+            and np.allclose(comp, np.array(g["compensated"], dtype=float), rtol=0, atol=1e-7)
+            and np.allclose(r["Err"][0], np.array(g["err"], dtype=float), rtol=0, atol=1e-7))
+
+
+@pytest.mark.parametrize("block_size", [0, 1, 2, 4])
+def test_worked_example_group_grid_from_current_values(golden_dir, block_size):
+    """Per-group grids are taken from the compensated values when the loop reaches the group: the
+    hand-worked d = 4, g = 2 example, where compensation moves group 1's maximum and the grid from
+    the original W would give a different code."""
+    g, Hd, w, bits, gs = _group_golden(golden_dir)
+    U = O.inverse_upper_cholesky(Hd)
+    np.testing.assert_allclose(np.diag(U), np.array(g["u_diag"], dtype=float), rtol=1e-14)
+    assert _check_group_golden(g, Hd, w, bits, gs, block_size)
+    np.testing.assert_array_equal(O.rtn_quantize(w, bits, gs)["codes"][0], np.array(g["rtn_codes"], dtype=int))
+
+
 @pytest.mark.parametrize("group_size", [0, 8])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_diagonal_hessian_reduces_to_rtn(bits, group_size):
@@ -278,3 +309,23 @@ def test_planted_mistakes_are_caught():
         except Exception:
             caught = True
         assert caught, name
+
+
+def test_planted_group_grid_from_original_w_is_caught(golden_dir, monkeypatch):
+    """Plant the mistake of taking each group's grid from the original W (rather than from the
+    compensated values at the group start) in the oracle, and check the hand-worked group pin fails.
+    The OBS recursion shares the grid routine, so it cannot see this mistake; the golden file can."""
+    import oracle.gptq_oracle as OM
+    g, Hd, w, bits, gs = _group_golden(golden_dir)
+    assert _check_group_golden(g, Hd, w, bits, gs, 2)
+    original = OM.grid_params
+    groups = [w[:, k:k + gs] for k in range(0, w.shape[1], gs)]
+    calls = {"n": 0}
+
+    def grid_from_original(xmin, xmax, b):
+        k = calls["n"] % len(groups)
+        calls["n"] += 1
+        return original(groups[k].min(axis=1), groups[k].max(axis=1), b)
+
+    monkeypatch.setattr(OM, "grid_params", grid_from_original)
+    assert not _check_group_golden(g, Hd, w, bits, gs, 2), "group grid from the original W"
