@@ -2,9 +2,10 @@
 """Throughput of the GPTQ layer solver on B200: quantized weights/s per layer, split by phase.
 
 One step = the whole hot path on one synthetic layer: H = 2 X^T X over the calibration tokens,
-dampening + U = chol(H^-1), the column loop with lazy block updates, and packing.  Inputs (X, W)
-are resident in HBM before timing; X (0.40 GB for the default layer) is larger than the 126 MB L2,
-so every step streams it from HBM.
+dampening + U = chol(H^-1), the column loop with lazy block updates, and packing.  The default layer
+is the largest that fits one GPU: the OPT-175B-like fc2 projection, W [12288, 49152], 262,144
+calibration tokens (X 25.8 GB, H and U 9.7 GB each).  Inputs (X, W) are resident in HBM before
+timing; X is larger than the 126 MB L2, so every step streams it from HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--layer NAME] [--impl ours|reference]
 
@@ -28,18 +29,19 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GPTQ quantized weights/sec & per-layer solve ms (1×B200), % of phase roofline"
-DEFAULT_LAYER = "opt125m_768x768"
+DEFAULT_LAYER = "opt175b_fc2_12288x49152"
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=30)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--layer", default=DEFAULT_LAYER)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--e2e-steps", type=int, default=None,
+                   help="end-to-end steps (default: 10, or 3 on layers whose step takes over 0.5 s)")
     return p.parse_args()
 
 
@@ -75,12 +77,38 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# fp32 FMA peak of the part: 148 SMs x 128 FMA lanes x 2 flops x clock (nominal max 1965 MHz)
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 / bf16 tensor throughput of the B200
 
 
-def fp32_peak_tflops(sm_mhz: float) -> float:
+def fp32_spec_tflops(sm_mhz: float) -> float:
+    """fp32 FMA peak from the part's unit counts: 148 SMs x 128 FMA lanes x 2 flops x clock."""
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def measure_fp32_fma_tflops(device, n: int = 8192, reps: int = 10) -> float:
+    """Measured fp32 FMA throughput: a cuBLAS fp32 GEMM (TF32 off, so it runs on the FMA units)
+    n^3, best of ``reps`` by CUDA events, in the way the bf16 tensor peak is measured."""
+    import torch
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        a = torch.randn(n, n, device=device)
+        b = torch.randn(n, n, device=device)
+        c = torch.empty(n, n, device=device)
+        for _ in range(3):
+            torch.matmul(a, b, out=c)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b, out=c)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b, c
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
 
 
 class ClockSampler:
@@ -158,15 +186,88 @@ def cores_info():
     return cores, blas
 
 
-def oracle_step(L, W64, X):
-    """One step of the oracle on the layer: the fp64 statement of the whole path (test infrastructure)."""
+FULL_ORACLE_MAX_D = 1024  # layers up to this width: the oracle runs the whole layer every step
+
+
+def oracle_full_step(L, W64, X):
+    """One step of the oracle on the whole layer: the fp64 statement of the path (test infrastructure)."""
     import numpy as np
     import oracle
     H = np.zeros((L.d, L.d))
     for t0 in range(0, L.n_tokens, 16384):
         oracle.hessian_accumulate(H, X[t0:t0 + 16384].double().numpy())
-    res = oracle.gptq_layer(W64, None, L.bits, L.group_size, L.block_size, L.damp, H=H)
-    return res
+    return oracle.gptq_layer(W64, None, L.bits, L.group_size, L.block_size, L.damp, H=H)
+
+
+class StagedOracle:
+    """The oracle on a bounded sample of a layer too large for it, extrapolated to the whole layer.
+
+    A step runs the oracle's phases, one at a time, on two sub-problems of the same layer: the first
+    n_s tokens, the first d1 and d2 channels and the first m_s rows.  Each phase's time is then scaled
+    to the full layer with a cost model:
+        Hessian   t = h N d^2                     (from the d2 run)
+        prepare   t = p d^3                       (from the d2 run)
+        quantize  t = q2 m d^2 + q1 m d           (two-point fit; lazy updates + column loop)
+        pack      t = k m d                       (from the d2 run)
+    Negative fitted coefficients (timing noise) are taken as 0.
+    """
+
+    def __init__(self, L, W, X_sample, d1=1024, d2=4096, m_s=512):
+        import numpy as np
+        self.L, self.d1, self.d2 = L, d1, d2
+        self.m_s = min(m_s, L.m)
+        self.n_s = X_sample.shape[0]
+        self.W = {dd: np.ascontiguousarray(W[:self.m_s, :dd].double().numpy()) for dd in (d1, d2)}
+        self.X = {dd: np.ascontiguousarray(X_sample[:, :dd].double().numpy()) for dd in (d1, d2)}
+        g = L.group_size
+        if g and (d1 % g or d2 % g):
+            raise ValueError("sample widths must hold whole groups")
+
+    def _phases(self, dd):
+        import oracle
+        L = self.L
+        t0 = time.perf_counter()
+        H = oracle.hessian(self.X[dd])
+        t1 = time.perf_counter()
+        U = oracle.inverse_upper_cholesky(oracle.dampen(H, L.damp))
+        t2 = time.perf_counter()
+        res = oracle.gptq_quantize(self.W[dd], U, L.bits, L.group_size, L.block_size)
+        t3 = time.perf_counter()
+        oracle.pack_codes(res["codes"], L.bits)
+        t4 = time.perf_counter()
+        return t1 - t0, t2 - t1, t3 - t2, t4 - t3
+
+    def step(self) -> float:
+        """Runs one sample; returns the extrapolated seconds of one full-layer oracle step."""
+        L, d1, d2, m_s = self.L, self.d1, self.d2, self.m_s
+        h1, p1, q1, k1 = self._phases(d1)
+        h2, p2, q2, k2 = self._phases(d2)
+
+        def fit(t_a, t_b, fa, fb, ga, gb):  # t = A f + B g through two points, A, B >= 0
+            det = fa * gb - fb * ga
+            A = max((t_a * gb - t_b * ga) / det, 0.0)
+            B = max((fa * t_b - fb * t_a) / det, 0.0)
+            return A, B
+
+        t_h = h2 * (L.n_tokens / self.n_s) * (L.d / d2) ** 2
+        t_p = p2 * (L.d / d2) ** 3
+        Q2, Q1 = fit(q1, q2, m_s * d1 ** 2, m_s * d2 ** 2, m_s * d1, m_s * d2)
+        t_q = Q2 * L.m * L.d ** 2 + Q1 * L.m * L.d
+        t_k = k2 * (L.m * L.d) / (m_s * d2)
+        self.last = {"hessian_s": t_h, "prepare_s": t_p, "quantize_s": t_q, "pack_s": t_k}
+        return t_h + t_p + t_q + t_k
+
+    def describe(self) -> str:
+        return (f"extrapolated: oracle phases timed on sub-problems of the {self.L.name} layer (first "
+                f"{self.n_s} tokens, first {self.d1} and {self.d2} channels, first {self.m_s} rows), scaled "
+                "to the full layer by per-phase cost models (Hessian N d^2, prepare d^3, pack m d from the wider "
+                "run; quantize m d^2 + m d fitted to both widths)")
+
+
+def oracle_sample_inputs(L, device="cpu"):
+    """The first chunk of X (2048 tokens) for the staged oracle."""
+    from post_weight_quantization_21_b200 import workloads as wl
+    return wl.make_x_chunk(L, 0, device).cpu()
 
 
 def run_reference(args, L):
@@ -174,23 +275,30 @@ def run_reference(args, L):
     if rank != 0:
         return
     from post_weight_quantization_21_b200 import workloads as wl
-    W64 = wl.make_w(L).double().numpy()
-    X = wl.make_x(L)
-    for _ in range(args.warmup):
-        oracle_step(L, W64, X)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(L, W64, X)
-    dt = (time.perf_counter() - t0) / args.steps
-    value = L.m * L.d / dt
     cores, blas = cores_info()
+    if L.d <= FULL_ORACLE_MAX_D:
+        W64 = wl.make_w(L).double().numpy()
+        X = wl.make_x(L)
+        for _ in range(args.warmup):
+            oracle_full_step(L, W64, X)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_full_step(L, W64, X)
+        dt = (time.perf_counter() - t0) / args.steps
+        sample = (f"the full {L.name} layer per step: fp64 H over all {L.n_tokens} tokens, U, column loop, "
+                  "pack (numpy/BLAS on the host cores)")
+    else:
+        st = StagedOracle(L, wl.make_w(L), oracle_sample_inputs(L))
+        for _ in range(args.warmup):
+            st.step()
+        dt = statistics.mean(st.step() for _ in range(args.steps))
+        sample = st.describe() + f"; one sample per step, mean of {args.steps}"
+    value = L.m * L.d / dt
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(L),
-            "cpu_baseline": {"value": value, "unit": "weights/s", "cores": blas, "kind": "oracle",
-                             "sample": f"the full {L.name} layer per step: fp64 H over all {L.n_tokens} tokens, "
-                                       "U, column loop, pack (numpy/BLAS on the host cores)"},
+            "cpu_baseline": {"value": value, "unit": "weights/s", "cores": blas, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -277,36 +385,37 @@ def main():
     value = world * L.m * L.d / (ms_per_step * 1e-3)
 
     # end to end through the host: pinned inputs in, packed codes + grids out, every step
-    W_h = torch.empty(solver.W.shape, dtype=solver.W.dtype).pin_memory()
-    X_h = torch.empty(solver.X.shape, dtype=solver.X.dtype).pin_memory()
+    W_h = torch.empty(solver.W.shape, dtype=solver.W.dtype, pin_memory=True)
+    X_h = torch.empty(solver.X.shape, dtype=solver.X.dtype, pin_memory=True)
     W_h.copy_(solver.W)
     X_h.copy_(solver.X)
     n_groups = 1 if L.group_size == 0 else L.d // L.group_size
-    out_p = torch.empty(L.m, L.d * L.bits // 32, dtype=torch.int32).pin_memory()
-    out_s = torch.empty(L.m, n_groups, dtype=torch.float32).pin_memory()
-    out_z = torch.empty(L.m, n_groups, dtype=torch.int32).pin_memory()
+    out_p = torch.empty(L.m, L.d * L.bits // 32, dtype=torch.int32, pin_memory=True)
+    out_s = torch.empty(L.m, n_groups, dtype=torch.float32, pin_memory=True)
+    out_z = torch.empty(L.m, n_groups, dtype=torch.int32, pin_memory=True)
+    e2e_steps = args.e2e_steps if args.e2e_steps is not None else (3 if ms_per_step > 500.0 else 10)
     solver.run_host(W_h, X_h, out_p, out_s, out_z, stream)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     e0.record(stream)
-    for _ in range(args.e2e_steps):
+    for _ in range(e2e_steps):
         solver.run_host(W_h, X_h, out_p, out_s, out_z, stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    solver.check_status(stream)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = slowest_rank_ms(e2e_ms, dev)
     h2d = W_h.numel() * W_h.element_size() + X_h.numel() * X_h.element_size()
     d2h = sum(t.numel() * t.element_size() for t in (out_p, out_s, out_z))
 
-    # roofline of each phase (algorithmic work per launch / measured time), against the pipe the
-    # library runs it on for this shape: bf16 tensor cores (Hessian), 3xTF32 tensor cores (block
-    # products of the blocked prepare, lazy block updates), or fp32 FMA units
-    sm_mhz = clk["sm_mhz"] if clk else 1965.0
+    # denominators: bf16 and HBM measured (MEASURED_PEAKS.json); fp32 FMA measured here by a cuBLAS
+    # fp32 GEMM; 3xTF32 derived from the measured bf16 figure and the nominal tf32/bf16 ratio
+    fp32_meas = measure_fp32_fma_tflops(dev)
     long_region = total_ms > 1000.0
     bf16_peak = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
-    fp32_peak = fp32_peak_tflops(1965.0)
+    fp32_peak = fp32_meas
     tf32x3_peak = bf16_peak * TF32_PER_BF16 / 3.0   # three tf32 MMAs per fp32-accurate product
     tc = g.gptq_tensor_core_phases(L.m, L.d, L.n_tokens, L.x_dtype, L.bits, L.group_size, L.block_size)
     h_flops = L.n_tokens * L.d * (L.d + 1)                 # symmetric half of 2 N d^2
@@ -315,6 +424,9 @@ def main():
     k_bytes = L.m * L.d * (1 + L.bits / 8)                  # pack: codes in, words out
     p_peak, p_pipe = (tf32x3_peak, "tensor(3xtf32)") if tc & g.GPTQ_TC_PREPARE else (fp32_peak, "fp32 FMA")
     q_peak, q_pipe = (tf32x3_peak, "tensor(3xtf32)") if tc & g.GPTQ_TC_LAZY else (fp32_peak, "fp32 FMA")
+    bf16_src = f"{pk['source']} bf16 {'sustained' if long_region else 'burst'}"
+    peak_src = {"tensor(bf16)": f"of {bf16_src}", "tensor(3xtf32)": f"derived: {bf16_src} x 1.1/2.25 / 3",
+                "fp32 FMA": "of measured fp32 GEMM", "hbm": f"of {pk['source']} HBM copy"}
     phases = {
         "hessian": {"ms": phase_ms[0], "tflops": h_flops / phase_ms[0] / 1e9,
                     "frac": h_flops / phase_ms[0] / 1e9 / bf16_peak, "pipe": "tensor(bf16)"},
@@ -325,6 +437,8 @@ def main():
         "pack": {"ms": phase_ms[3], "gbs": k_bytes / phase_ms[3] / 1e6,
                  "frac": k_bytes / phase_ms[3] / 1e6 / pk["hbm_gbs"], "pipe": "hbm"},
     }
+    for ph in phases.values():
+        ph["peak_source"] = peak_src[ph["pipe"]]
     roof_ms = (h_flops / bf16_peak / 1e9 + p_flops / p_peak / 1e9 + q_flops / q_peak / 1e9
                + k_bytes / pk["hbm_gbs"] / 1e6)
     # the same sum with prepare and quantize bounded by the fp32 FMA units (their roofline before
@@ -332,40 +446,71 @@ def main():
     roof_fp32_ms = (h_flops / bf16_peak / 1e9 + p_flops / fp32_peak / 1e9 + q_flops / fp32_peak / 1e9
                     + k_bytes / pk["hbm_gbs"] / 1e6)
     h_tflops = h_flops / phase_ms[0] / 1e9
-    roofline = {"bound": "tensor", "kernel": "hessian (A1)", "achieved": h_tflops, "peak": bf16_peak,
-                "unit": "TFLOP/s", "frac": h_tflops / bf16_peak,
-                "peak_source": f"{pk['source']} bf16 {'sustained' if long_region else 'burst'}",
-                "algorithmic": f"N*d*(d+1) = {h_flops:.4g} flop per launch (N={L.n_tokens}, d={L.d})",
-                "traffic": kernel_traffic("hessian_" + L.name, hessian_sources())}
+    roof_hessian = {"bound": "tensor", "kernel": "hessian_tc_kernel (A1, one launch per step)",
+                    "achieved": h_tflops, "peak": bf16_peak, "unit": "TFLOP/s", "frac": h_tflops / bf16_peak,
+                    "peak_source": bf16_src,
+                    "algorithmic": f"N*d*(d+1) = {h_flops:.4g} flop per launch (N={L.n_tokens}, d={L.d})",
+                    "traffic": kernel_traffic("hessian_" + L.name, hessian_sources())}
+    # the phase that takes the largest share of the step
+    work = {"hessian": (h_flops, "N*d*(d+1) flop"), "prepare": (p_flops, "2/3 d^3 flop"),
+            "quantize": (q_flops, "m*d^2 flop"), "pack": (k_bytes, "m*d*(1+b/8) byte")}
+    top = max(phases, key=lambda k: phases[k]["ms"])
+    if top == "hessian":
+        roofline = roof_hessian
+    else:
+        ph = phases[top]
+        hbm = ph["pipe"] == "hbm"
+        achieved = ph["gbs"] if hbm else ph["tflops"]
+        peak = pk["hbm_gbs"] if hbm else {"tensor(3xtf32)": tf32x3_peak, "fp32 FMA": fp32_peak}[ph["pipe"]]
+        kernels = {"prepare": "prepare phase (A2+A3): factor_kernel, tf32x3_gemm_kernel (trsm/syrk/trtri), "
+                              "diag_mean, reverse_damp, leaf_copy, rotate" if tc & g.GPTQ_TC_PREPARE
+                              else "prepare phase (A2+A3): prepare_kernel (one cooperative launch)",
+                   "quantize": "quantize phase (A4-A6): column loop + lazy block updates",
+                   "pack": "pack_kernel (A7)"}[top]
+        roofline = {"bound": "hbm" if hbm else "tensor" if ph["pipe"].startswith("tensor") else "alu",
+                    "kernel": kernels, "achieved": achieved, "peak": peak, "unit": "GB/s" if hbm else "TFLOP/s",
+                    "frac": achieved / peak, "peak_source": ph["peak_source"],
+                    "algorithmic": f"{work[top][1]} = {work[top][0]:.4g} per step (one phase = one unit)",
+                    "traffic": None}
 
     line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(L),
             "e2e": {"value": world * L.m * L.d / (e2e_ms * 1e-3), "unit": "weights/s", "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": int(launches), "roofline": roofline, "phases": phases,
-            "phase_roofline_ms": roof_ms, "end_to_end_roofline_frac": roof_ms / ms_per_step,
+                    "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches), "roofline": roofline, "roofline_hessian": roof_hessian,
+            "phases": phases, "phase_roofline_ms": roof_ms, "end_to_end_roofline_frac": roof_ms / ms_per_step,
             "peaks": {"bf16_tflops": bf16_peak, "tf32x3_tflops": tf32x3_peak, "fp32_fma_tflops": fp32_peak,
-                      "hbm_gbs": pk["hbm_gbs"],
-                      "note": "bf16 and HBM measured; tf32 = bf16 x 1.1/2.25 (nominal ratio) / 3 MMAs; fp32 FMA = "
-                              "148 SMs x 128 lanes x 2 x 1965 MHz"},
+                      "fp32_fma_spec_tflops_at_max_clock": fp32_spec_tflops(1965.0), "hbm_gbs": pk["hbm_gbs"],
+                      "note": "bf16 and HBM measured (MEASURED_PEAKS.json); fp32 FMA measured in this run "
+                              "(cuBLAS fp32 GEMM 8192^3, TF32 off, best of 10); tf32 = bf16 x 1.1/2.25 "
+                              "(nominal ratio) / 3 MMAs"},
             "end_to_end_roofline_frac_fp32_pipes": roof_fp32_ms / ms_per_step,
             "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        W64 = W_h.double().numpy()
-        X = X_h
         cores, blas = cores_info()
         t0 = time.perf_counter()
-        n = 0
-        while True:
-            oracle_step(L, W64, X)
-            n += 1
-            if time.perf_counter() - t0 > 10.0 or n >= 20:
-                break
-        dt = (time.perf_counter() - t0) / n
+        n, times = 0, []
+        if L.d <= FULL_ORACLE_MAX_D:
+            W64 = W_h.double().numpy()
+            while True:
+                oracle_full_step(L, W64, X_h)
+                n += 1
+                if time.perf_counter() - t0 > 10.0 or n >= 20:
+                    break
+            dt = (time.perf_counter() - t0) / n
+            sample = f"{n} full oracle step(s) of the {L.name} layer (fp64, all {L.n_tokens} tokens), {dt:.2f} s each"
+        else:
+            st = StagedOracle(L, W_h, X_h[:2048])
+            while True:
+                times.append(st.step())
+                n += 1
+                if time.perf_counter() - t0 > 10.0 or n >= 20:
+                    break
+            dt = statistics.mean(times)
+            sample = st.describe() + f"; {n} sample(s) in {time.perf_counter() - t0:.1f} s"
         line["cpu_baseline"] = {"value": L.m * L.d / dt, "unit": "weights/s", "cores": blas, "kind": "oracle",
-                                "sample": f"{n} full oracle step(s) of the {L.name} layer (fp64, all "
-                                          f"{L.n_tokens} tokens), {dt:.2f} s each"}
+                                "sample": sample, "seconds_per_layer": dt}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -86,7 +86,9 @@ typedef struct {
  *   H          [d, d] fp32 row-major.  On return the upper triangle (j >= i) holds the result; the
  *              strict lower triangle is left unspecified.
  *   workspace  >= gptq_hessian_workspace_size(n_tokens, d, x_dtype) bytes, 256-byte aligned.
- *   dev_status int32[2] device status word (written only on a device-side failure).
+ *   dev_status int32[2] device status word: cleared at the start of a call with accumulate = 0 (a
+ *              chunked sequence keeps the first failure of any of its calls); GPTQ_ERR_TIMEOUT if a
+ *              bounded device wait gave up.
  *   Requires d % 8 == 0, n_tokens >= 0 (0 tokens gives H = 0 or leaves H unchanged).
  * ------------------------------------------------------------------------------------------ */
 GPTQ_API gptq_status gptq_hessian_accumulate(const void* X, int32_t x_dtype, int64_t n_tokens, int64_t d,
@@ -131,7 +133,9 @@ GPTQ_API size_t gptq_prepare_workspace_size(int64_t d);
  *   H, d, damp, U, dev_status, stream: as for gptq_prepare_uinv (U is still caller memory).
  *   d > GPTQ_PREPARE_STATIC_MAX_D returns GPTQ_ERR_WORKSPACE and enqueues nothing.
  *   The first call on each device looks up the array's device address (a host-side runtime call,
- *   with that device current); make that first call before any stream capture.
+ *   with that device current); make that first call before any stream capture.  The address is
+ *   cached with the id of the device's context and looked up again when the context changes (after
+ *   cudaDeviceReset, say): make the first call after such a change before any stream capture too.
  *   All calls share the one array and it keeps the last call's contents (each call clears the parts
  *   that must start at zero).  Calls that overlap on the GPU, on any streams, race on it: order them.
  *   It creates no CUDA objects: above d = 1024 every launch goes to `stream` (no look-ahead stream).
@@ -148,8 +152,11 @@ GPTQ_API gptq_status gptq_prepare_uinv_static(const float* H, int64_t d, float d
  * + zero, 0, 2^b-1); err = (w_i - scale*(q_i - zero)) / U_ii; W[:, j] -= err * U[i, j] for the
  * remaining columns j of the block at once, and for the columns after the block once per block.
  * Grid: asymmetric min/max over the row (per-row, from the original W) or over the group's current
- * values when the loop reaches the group (per-group), the range widened to contain 0.  The grid
- * decisions (zero point and codes) use IEEE fp32 division and round-half-to-even.
+ * values when the loop reaches the group (per-group), the range widened to contain 0.  The scale and
+ * the zero point are IEEE fp32 divisions, rounded half-to-even for the zero point.  Each code's
+ * quotient w_i / scale is formed as the fp32 product of w_i and the IEEE fp32 reciprocal of the scale,
+ * then rounded half-to-even; it differs from the IEEE quotient by about one ulp at most, so a code can
+ * be one level away from the division's only when the quotient is within a few ulps of a half-integer.
  *
  *   W          [m, d] row-major, dtype w_dtype (FP16, BF16 or FP32); read only.
  *   U          [d, d] fp32 upper factor from gptq_prepare_uinv (strict lower part ignored).

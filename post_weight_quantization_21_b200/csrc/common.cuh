@@ -48,9 +48,11 @@ template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // Asymmetric min/max grid: the range widened to contain 0, an empty range becomes [-1, 1];
-// scale = (hi - lo) / maxq in IEEE fp32, rscale = IEEE fp32 reciprocal of scale, and
-// zero = rint(-lo * rscale).  Quotients that decide an integer are always formed as x * rscale
-// (IEEE fp32 product, not contracted into an FMA).
+// scale = (hi - lo) / maxq and zero = rint(-lo / scale), both quotients IEEE fp32 divisions (once per
+// grid); rscale = IEEE fp32 reciprocal of scale.  The column loops form each code's quotient as the
+// IEEE fp32 product x * rscale (not contracted into an FMA) instead of the division x / scale: the two
+// differ by at most about one ulp, so a code can differ from the division's by one level only when
+// the quotient lies within a few ulps of a half-integer.
 // Round to the nearest integer, ties to even, with two fp32 adds on the FMA pipe: adding 1.5 * 2^23
 // moves |x| < 2^22 into [2^23, 2^24), where the spacing of floats is 1, so the addition itself rounds.
 // Equal to rintf(x) for |x| < 2^22; larger magnitudes come out at least 2^22 - 1 in magnitude, beyond
@@ -70,7 +72,7 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, 
   }
   scale = __fdiv_rn(hi - lo, maxq);
   rscale = __frcp_rn(scale);
-  zero = rintf(__fmul_rn(-lo, rscale));
+  zero = rintf(__fdiv_rn(-lo, scale));
 }
 
 __device__ __forceinline__ float warp_min(float v) {

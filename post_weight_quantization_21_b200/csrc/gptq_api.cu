@@ -50,7 +50,7 @@ int32_t gptq_tensor_core_phases(int64_t m, int64_t d, int64_t n_tokens, int32_t 
   int32_t mask = 0;
   if (gptq::hessian_tc_supported(n_tokens, d, x_dtype)) mask |= GPTQ_TC_HESSIAN;
   if (gptq::prepare_uses_tensor_cores(d)) mask |= GPTQ_TC_PREPARE;
-  if (!gptq::quantize_fused(m, d) && !(cfg->flags & GPTQ_FLAG_FP32_FMA)) mask |= GPTQ_TC_LAZY;
+  if (gptq::quantize_lazy_on_tensor_cores(m, d, cfg->flags)) mask |= GPTQ_TC_LAZY;
   return mask;
 }
 
@@ -80,13 +80,15 @@ gptq_status gptq_hessian_accumulate(const void* X, int32_t x_dtype, int64_t n_to
   if (!aligned(X, 16) || !aligned(H, 16) || !aligned(dev_status, 4)) return GPTQ_ERR_ARG;
   if (accumulate != 0 && accumulate != 1) return GPTQ_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t need = n_tokens ? gptq::hessian_workspace(n_tokens, d, x_dtype) : 0;
+  if (need && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
+    return GPTQ_ERR_WORKSPACE;
+  // a fresh sum starts with a clear status word; accumulating calls keep what earlier calls recorded
+  if (!accumulate) GPTQ_CUDA_TRY(cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s));
   if (n_tokens == 0) {
     if (!accumulate) GPTQ_CUDA_TRY(cudaMemsetAsync(H, 0, (size_t)d * d * sizeof(float), s));
     return GPTQ_OK;
   }
-  const size_t need = gptq::hessian_workspace(n_tokens, d, x_dtype);
-  if (need && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
-    return GPTQ_ERR_WORKSPACE;
   return gptq::hessian_launch(X, x_dtype, n_tokens, d, H, scale, accumulate, dev_status, workspace, s);
 }
 

@@ -49,6 +49,8 @@ size_t prepare_blocked_workspace(int64_t d);
 gptq_status prepare_blocked_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
                                    void* workspace, cudaStream_t stream, bool lookahead);
 size_t prepare_workspace(int64_t d);
+// the blocked path's tile products run as 3xTF32 tensor-core products; the launch takes exactly this
+// path or fails
 bool prepare_uses_tensor_cores(int64_t d);
 gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
                            void* workspace, cudaStream_t stream, bool lookahead = true);
@@ -59,6 +61,9 @@ gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* 
 // A4 - A6
 size_t quantize_workspace(int64_t m, int64_t d, int block_size);
 bool quantize_fused(int64_t m, int64_t d);  // one launch per layer (U resident in L2) rather than launches per block
+// the lazy block updates run as 3xTF32 tensor-core products (the per-block path without GPTQ_FLAG_FP32_FMA,
+// with a tile count that fits 32 bits); the launch takes exactly this path or fails
+bool quantize_lazy_on_tensor_cores(int64_t m, int64_t d, uint32_t flags);
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
                             int32_t* status, void* workspace, cudaStream_t stream);

@@ -26,6 +26,9 @@
 //   phase R   U = J Y J: lower block triangle -> upper, strict lower part zeroed.
 #include <math.h>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -517,21 +520,57 @@ static __device__ __align__(256) unsigned char g_prepare_scratch[kStaticScratchB
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_address[kMaxDevices] = {};
+struct ScratchAddress {
+  unsigned long long ctx_id;  // the context the address belongs to
+  void* addr;
+};
+ScratchAddress g_scratch_address[kMaxDevices] = {};
 
-// Device address of g_prepare_scratch on the current device; looked up once per device, with that
-// device current.  Host code must not use the symbol itself: it is a host-side stand-in.
+// Unique id of the calling thread's current CUDA context (through the runtime's driver entry points,
+// no link against libcuda); false when no context is current or the driver lacks the calls.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_prepare_scratch in the current device's context.  Host code must not use the
+// symbol itself: it is a host-side stand-in.  The address is looked up with that device current and
+// cached per device together with the context's id; when the context changes (the device was reset,
+// or its primary context released and made again, which reloads the module) it is looked up again.
 gptq_status static_scratch(void** out) {
   int dev = 0;
   GPTQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return GPTQ_ERR_CUDA;
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_address[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_prepare_scratch) != cudaSuccess || p == nullptr) return GPTQ_ERR_CUDA;
-    g_scratch_address[dev] = p;
+  ScratchAddress& c = g_scratch_address[dev];
+  if (have_id && c.addr != nullptr && c.ctx_id == id) {
+    *out = c.addr;
+    return GPTQ_OK;
   }
-  *out = g_scratch_address[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_prepare_scratch) != cudaSuccess || p == nullptr) return GPTQ_ERR_CUDA;
+  if (!have_id) have_id = current_context_id(&id);  // the lookup makes the device's context current
+  c.ctx_id = have_id ? id : 0;
+  c.addr = have_id ? p : nullptr;  // without a context id nothing is cached: the next call looks up again
+  *out = p;
   return GPTQ_OK;
 }
 }  // namespace

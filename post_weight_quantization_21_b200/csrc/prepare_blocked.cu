@@ -500,7 +500,10 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
   GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFactorSmem));
   TcMaps maps;
-  const bool tc = tc_maps(maps, U, side, d, D);
+  const bool tc = prepare_uses_tensor_cores(d);
+  // U is 16-byte aligned (checked by the entry points), the scratch 256-byte aligned and d % 4 == 0 on
+  // this path, so the maps encode unless the driver call itself fails
+  if (tc && !tc_maps(maps, U, side, d, D)) return GPTQ_ERR_CUDA;
   std::unique_lock<std::mutex> hold(g_lookahead_mu, std::defer_lock);
   LookAhead* la = nullptr;
   if (lookahead && dev < 64) {

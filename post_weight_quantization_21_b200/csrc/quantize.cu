@@ -592,10 +592,12 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(colloop_kernel<C4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid_rows = (int)((m + loop_rows - 1) / loop_rows);
   CUtensorMap mErr, mU, mW;
-  // the tensor-core update numbers its 128x128 tiles with 32-bit ints
-  const bool tiles_fit = ((m + 127) / 128) * (int64_t)((d + 127) / 128) <= 0x7fffffff;
-  const bool tc = !fma && status != nullptr && tiles_fit && tf32x3_map(&mErr, err, m, B, B, 128) &&
-                  tf32x3_map(&mU, U, d, d, d, 32, true) && tf32x3_map(&mW, ww, m, d, d, 32);
+  const bool tc = quantize_lazy_on_tensor_cores(m, d, fma ? GPTQ_FLAG_FP32_FMA : 0u);
+  // every base is 16-byte aligned and every row stride a multiple of 16 bytes here (d % 32 == 0), so
+  // the maps encode unless the driver call itself fails
+  if (tc && !(tf32x3_map(&mErr, err, m, B, B, 128) && tf32x3_map(&mU, U, d, d, d, 32, true) &&
+              tf32x3_map(&mW, ww, m, d, d, 32)))
+    return GPTQ_ERR_CUDA;
   Tf32x3Args g{};
   g.kind = kGemmLazy;
   g.epi = kEpiSub;
@@ -664,6 +666,12 @@ size_t quantize_workspace(int64_t m, int64_t d, int block_size) {
 // from L2 for only 8 rows); with many rows the per-block launches run the lazy update as one large
 // GEMM across all rows instead.
 bool quantize_fused(int64_t m, int64_t d) { return d <= 4096 && m <= 2048; }
+
+bool quantize_lazy_on_tensor_cores(int64_t m, int64_t d, uint32_t flags) {
+  // the tensor-core update numbers its 128x128 tiles with 32-bit ints
+  const bool tiles_fit = ((m + 127) / 128) * ((d + 127) / 128) <= 0x7fffffff;
+  return !quantize_fused(m, d) && !(flags & GPTQ_FLAG_FP32_FMA) && tiles_fit;
+}
 
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d64, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,

@@ -34,3 +34,19 @@ def read_golden(path):
     if rows:
         out["rows"] = rows
     return out
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Code mismatches of every GPU parity comparison with the oracle (near-tie decisions and the
+    trajectories that follow them), one line per comparison."""
+    sup = sys.modules.get("gpu_support")
+    log = getattr(sup, "PARITY_LOG", None)
+    if not log:
+        return
+    terminalreporter.section("code parity against the oracle")
+    for label, st in log:
+        terminalreporter.write_line(
+            f"{label}: agree {st['agree']:.6f}, mismatched codes {st['mismatches']}"
+            + (f", rows diverged {st['rows_diverged']}, max level diff {st['max_level_diff']}"
+               if "rows_diverged" in st else "")
+            + (f", E rel {st['E_rel']:.2e}" if "E_rel" in st else ""))

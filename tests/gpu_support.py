@@ -13,6 +13,10 @@ SCALE_REL = 1e-5         # scales relative error (per-row: all rows; per-group: 
 E_REL = 0.02             # layer reconstruction error, relative
 
 
+# every compare_quantization call appends (label, stats) here; the session summary prints them
+PARITY_LOG: list[tuple[str, dict]] = []
+
+
 def dev():
     return torch.device("cuda", 0)
 
@@ -88,6 +92,8 @@ def compare_quantization(gpu, ref, group_size, W=None, H=None, E_ref=None, label
     rc, rs, rz = ref["codes"], ref["scales"], ref["zeros"]
     diff = codes - rc
     agree = float(np.mean(diff == 0))
+    if agree < CODES_MIN_AGREE:
+        PARITY_LOG.append((label, {"agree": agree, "mismatches": int(np.sum(diff != 0)), "failed": True}))
     assert agree >= CODES_MIN_AGREE, f"{label}: codes agree {agree:.5f}"
     m, d = codes.shape
     bad_rows = (diff != 0).any(axis=1)
@@ -119,6 +125,7 @@ def compare_quantization(gpu, ref, group_size, W=None, H=None, E_ref=None, label
         checked = int(upto.sum())
     stats = {"agree": agree, "mismatches": int(np.sum(diff != 0)), "rows_diverged": int(bad_rows.sum()),
              "max_level_diff": int(np.abs(diff).max()), "grids_checked": checked}
+    PARITY_LOG.append((label, stats))
     if W is not None and H is not None:
         import oracle
         E_gpu = oracle.reconstruction_error(W, dequant(codes, scales, zeros, group_size), H)

@@ -151,6 +151,65 @@ def test_quantize_per_block_paths(m, d, bits, gs, B, flags):
     S.compare_quantization(gpu, ref, gs, W.double().numpy(), H, label=f"{m}x{d} b{bits} g{gs} B{B} f{flags}")
 
 
+# Edge cases of the method on both quantize paths: a zero row of W (flat range, grid [-1, 1]), a zero
+# group, an all-positive row (range widened to 0), outlier weights (x10) under group grids, dead input
+# channels (H_ii = 0: only the damping keeps Hd positive definite), 2-bit groups, a group of 128
+# spanning several blocks of 32 or 64.
+EDGE_CASES = [
+    # m, d, bits, group, block
+    (64, 512, 2, 128, 128),     # fused path
+    (64, 512, 4, 128, 32),
+    (2100, 512, 2, 128, 128),   # per-block path (many rows)
+    (2100, 512, 4, 128, 32),
+    (40, 4352, 3, 128, 64),     # per-block path (wide)
+]
+
+
+def _edge_inputs(m, d, seed):
+    gen = torch.Generator().manual_seed(seed)
+    X = _x(4 * d, d, torch.float64, seed=seed)
+    dead = [3, 77, d // 2, d - 1]
+    X[:, dead] = 0.0
+    W = torch.randn(m, d, generator=gen) * 0.02
+    k = max(1, (m * d) // 200)                    # 0.5 % of the entries x10
+    idx = torch.randperm(m * d, generator=gen)[:k]
+    W.view(-1)[idx] *= 10.0
+    W[5] = 0.0                                    # zero row
+    W[7, 128:256] = 0.0                           # zero group (and a zero stretch of a per-row grid)
+    W[9] = W[9].abs()                             # all-positive row
+    return X, W.half(), dead
+
+
+@pytest.mark.parametrize("m,d,bits,gs,B", EDGE_CASES)
+def test_quantize_edge_cases(m, d, bits, gs, B):
+    X, W, dead = _edge_inputs(m, d, seed=m + d + bits + B)
+    H = oracle.hessian(X.numpy())
+    assert np.all(np.diag(H)[dead] == 0.0)
+    U = oracle.inverse_upper_cholesky(oracle.dampen(H, 0.01))
+    U32 = np.ascontiguousarray(U, dtype=np.float32)
+    ref = oracle.gptq_quantize(W.double().numpy(), U32.astype(np.float64), bits, gs, B)
+    gpu = S.quantize(W.to(S.dev()), torch.from_numpy(U32).to(S.dev()), bits, gs, B)
+    S.compare_quantization(gpu, ref, gs, W.double().numpy(), H, label=f"edge {m}x{d} b{bits} g{gs} B{B}")
+    # the zero row: every code is the zero point, the grid is [-1, 1]
+    assert np.all(gpu[0][5] == gpu[2][5][0]) and np.all(gpu[2][5] == ref["zeros"][5])
+    np.testing.assert_allclose(gpu[1][5], np.float32(2.0) / np.float32(2 ** bits - 1), rtol=1e-7)
+
+
+@pytest.mark.parametrize("d", [768, 2048])
+def test_prepare_dead_channels(d):
+    X, _, dead = _edge_inputs(8, d, seed=d)
+    H = oracle.hessian(X.numpy())
+    Hd = oracle.dampen(H, 0.01)
+    Uref = oracle.inverse_upper_cholesky(Hd)
+    U = S.prepare(torch.from_numpy(H).float().to(S.dev())).cpu().numpy().astype(np.float64)
+    rel = np.linalg.norm(U - Uref) / np.linalg.norm(Uref)
+    kappa = np.linalg.cond(Hd)
+    assert rel <= max(1e-5, 10 * kappa * 6e-8), (rel, kappa)
+    # the last channel is dead: its row and column of Hd are lambda e_(d-1), so U_(d-1,d-1) = lambda^-1/2
+    lam = 0.01 * np.mean(np.diag(H))
+    np.testing.assert_allclose(U[d - 1, d - 1], lam ** -0.5, rtol=1e-5)
+
+
 def test_quantize_fp32_and_bf16_weights():
     d, m = 256, 32
     X = _x(4 * d, d, torch.float64, seed=3)

@@ -3,8 +3,10 @@
 Callers that cannot allocate device memory (a plugin whose host application owns every buffer, a
 path where no allocator may run) use this variant: its scratch is a fixed array inside the library.
 The test calls it through the C ABI twice in a row and compares each result with the workspace
-entry point's on the same input; it also checks that an order above the array's limit is refused
-before any work is enqueued.  This file is collected last on purpose.
+entry point's on the same input, on both prepare paths: the one-launch kernel (d <= 1024) and the
+blocked path above it, with tensor-core tiles (d = 2048) and fp32 tiles (d = 1030, rows not 16-byte
+aligned).  Each result is also held to the oracle's U.  It also checks that an order above the
+array's limit is refused before any work is enqueued.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -12,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import post_weight_quantization_21_b200 as g
 
 pytestmark = pytest.mark.gpu
@@ -23,13 +26,19 @@ def _spd_hessian(d, seed):
     gen = torch.Generator().manual_seed(seed)
     X = torch.randn(4 * d, d, generator=gen, dtype=torch.float64)
     X = X @ (torch.randn(d, d, generator=gen, dtype=torch.float64) / d ** 0.5)
-    return (2.0 * X.T @ X).float().cuda()
+    return 2.0 * X.T @ X
 
 
-@pytest.mark.parametrize("d", [200, 768])
+# 200, 768: one-launch kernel; 2048: blocked path, tensor-core tiles; 1030: blocked path, fp32 tiles
+@pytest.mark.parametrize("d", [200, 768, 2048, 1030])
 def test_static_prepare_matches_workspace_prepare(d):
     lib = g.lib()
-    H = _spd_hessian(d, seed=d)
+    H64 = _spd_hessian(d, seed=d)
+    H = H64.float().cuda()
+    Hd = oracle.dampen(H.double().cpu().numpy(), 0.01)
+    Uo = oracle.inverse_upper_cholesky(Hd)
+    kappa = np.linalg.cond(Hd)
+    o_tol = max(1e-5, 10 * kappa * 6e-8)  # the prepare parity tests' bound against the oracle
     stream = torch.cuda.current_stream().cuda_stream
     status = torch.zeros(4, dtype=torch.int32, device="cuda")
     ws = torch.empty(g.gptq_prepare_workspace_size(d), dtype=torch.uint8, device="cuda")
@@ -49,6 +58,8 @@ def test_static_prepare_matches_workspace_prepare(d):
         rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
         assert rel <= U_REL, rel
         assert np.all(np.tril(got, -1) == 0.0)
+        rel_o = np.linalg.norm(got - Uo) / np.linalg.norm(Uo)
+        assert rel_o <= o_tol, (rel_o, kappa)
 
 
 def test_static_prepare_refuses_orders_above_its_scratch():
