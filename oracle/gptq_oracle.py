@@ -46,6 +46,7 @@ __all__ = [
     "inverse_upper_cholesky_reversed", "grid_params", "quantize_codes", "dequantize",
     "gptq_quantize", "rtn_quantize", "obs_quantize", "conditional_ls_values",
     "bruteforce_best_codes", "reconstruction_error", "pack_codes", "unpack_codes", "gptq_layer",
+    "act_order_permutation", "gptq_quantize_act_order", "act_order_group_index",
 ]
 
 
@@ -232,27 +233,34 @@ def rtn_quantize(W, bits: int, group_size: int = 0):
 #   W_F -= (w_i - q_i) / Hinv[i,i] * Hinv[i, F];   Hinv <- Hinv - Hinv[:, i] Hinv[i, :] / Hinv[i,i].
 # Used only to pin the Cholesky form (small d).
 # --------------------------------------------------------------------------------------------
-def obs_quantize(W, Hd, bits: int, group_size: int = 0):
+def obs_quantize(W, Hd, bits: int, group_size: int = 0, order=None):
+    """``order`` (default: natural) is the sequence in which columns are quantized; the recursion
+    needs no permuted matrices: it removes each quantized column from the free set F directly.  A
+    group is ``group_size`` consecutive steps of the order; its grid comes from the current values of
+    the group's columns at its first step."""
     Wc = np.array(W, dtype=np.float64)
     m, d = Wc.shape
+    order = np.arange(d) if order is None else np.asarray(order)
     Hinv = np.linalg.inv(np.asarray(Hd, dtype=np.float64))
     n_groups = 1 if group_size == 0 else d // group_size
     scales = np.zeros((m, n_groups), dtype=np.float32)
     zeros = np.zeros((m, n_groups), dtype=np.int64)
     codes = np.zeros((m, d), dtype=np.int64)
+    free = np.ones(d, dtype=bool)
     if group_size == 0:
         s, z = grid_params(Wc.min(axis=1), Wc.max(axis=1), bits)
         scales[:, 0], zeros[:, 0] = s, z
-    for i in range(d):
-        if group_size and i % group_size == 0:
-            cols = Wc[:, i:i + group_size]
+    for k, i in enumerate(order):
+        if group_size and k % group_size == 0:
+            cols = Wc[:, order[k:k + group_size]]
             s, z = grid_params(cols.min(axis=1), cols.max(axis=1), bits)
-            scales[:, i // group_size], zeros[:, i // group_size] = s, z
-        g = i // group_size if group_size else 0
+            scales[:, k // group_size], zeros[:, k // group_size] = s, z
+        g = k // group_size if group_size else 0
         q = quantize_codes(Wc[:, i], scales[:, g], zeros[:, g], bits)
         delta = Wc[:, i] - dequantize(q, scales[:, g], zeros[:, g])
         hii = Hinv[i, i]
-        Wc[:, i + 1:] -= np.outer(delta / hii, Hinv[i, i + 1:])
+        free[i] = False
+        Wc[:, free] -= np.outer(delta / hii, Hinv[i, free])
         Hinv = Hinv - np.outer(Hinv[:, i], Hinv[i, :]) / hii
         codes[:, i] = q
     return {"codes": codes, "scales": scales, "zeros": zeros}
@@ -323,6 +331,47 @@ def unpack_codes(packed, bits: int, d: int) -> np.ndarray:
             v = v | (p[:, w + 1] << np.uint64(32 - sh))
         out[:, j] = (v & mask).astype(np.int64)
     return out
+
+
+# --------------------------------------------------------------------------------------------
+# Act-order ("desc_act").  [ZLY] 实践指南 lists desc_act (off by default); [CSDN] 关键参数说明 lists
+# it among the quantizer's settings.  The pages do not define the order beyond its name ("sort by
+# activation"); reading: the columns are quantized in descending order of diag(H) (the channels with
+# the largest calibration activations first), ties in column order.  The method itself is unchanged:
+# it runs on the permuted problem (H -> P H P^T, W -> W P^T), and the codes are put back in the
+# original column order.  Groups are consecutive columns of the quantization order, so group k
+# holds the original columns perm[k*g : (k+1)*g].
+# --------------------------------------------------------------------------------------------
+def act_order_permutation(H) -> np.ndarray:
+    """perm[i] = the original column quantized at step i: descending diag(H), ties by column index."""
+    diag = np.diag(np.asarray(H, dtype=np.float64))
+    return np.argsort(-diag, kind="stable")
+
+
+def act_order_group_index(perm, group_size: int) -> np.ndarray:
+    """Group of each original column: the step at which it is quantized, divided by the group size."""
+    perm = np.asarray(perm)
+    step = np.empty_like(perm)
+    step[perm] = np.arange(perm.shape[0])
+    return step // group_size if group_size else np.zeros_like(step)
+
+
+def gptq_quantize_act_order(W, H, bits: int, group_size: int = 0, block_size: int = 0, damp: float = 0.01,
+                            perm=None):
+    """The column loop in act-order.  Returns codes and Wq in the original column order, the grids of
+    the groups of the quantization order, perm, the group index of every original column, and the
+    factor U of the permuted dampened Hessian."""
+    H = np.asarray(H, dtype=np.float64)
+    if perm is None:
+        perm = act_order_permutation(H)
+    perm = np.asarray(perm)
+    U = inverse_upper_cholesky(dampen(H[np.ix_(perm, perm)], damp))
+    r = gptq_quantize(np.asarray(W, dtype=np.float64)[:, perm], U, bits, group_size, block_size)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.shape[0])
+    return {"codes": r["codes"][:, inv], "Wq": r["Wq"][:, inv], "scales": r["scales"], "zeros": r["zeros"],
+            "perm": perm, "g_idx": act_order_group_index(perm, group_size), "U": U,
+            "codes_in_order": r["codes"]}
 
 
 # --------------------------------------------------------------------------------------------

@@ -283,6 +283,81 @@ def test_pack_roundtrip(bits):
     np.testing.assert_array_equal(O.unpack_codes(p, bits, 96), codes)
 
 
+# ------------------------------------------------------------------------------------ act-order
+def _act_golden(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "worked_example_act_order.txt"))
+    return g, np.array(g["hd"], dtype=float).reshape(3, 3), np.array(g["w"], dtype=float)[None, :], int(g["bits"][0])
+
+
+def _act_golden_holds(golden_dir, fn=None):
+    g, Hd, w, bits = _act_golden(golden_dir)
+    fn = fn or (lambda w, Hd, bits: O.gptq_quantize_act_order(w, Hd, bits, damp=0.0))
+    r = fn(w, Hd, bits)
+    return (np.array_equal(r["perm"], np.array(g["perm"], dtype=int))
+            and np.array_equal(r["codes"][0], np.array(g["codes"], dtype=int)))
+
+
+def test_act_order_worked_example(golden_dir):
+    g, Hd, w, bits = _act_golden(golden_dir)
+    r = O.gptq_quantize_act_order(w, Hd, bits, damp=0.0)  # Hd is used as the damped matrix directly
+    np.testing.assert_array_equal(r["perm"], np.array(g["perm"], dtype=int))
+    np.testing.assert_array_equal(r["codes"][0], np.array(g["codes"], dtype=int))
+    U = r["U"]
+    rin = O.gptq_quantize(w[:, r["perm"]], U, bits)
+    comp = rin["Wq"][0] + rin["Err"][0] * np.diag(U)
+    np.testing.assert_allclose(comp, np.array(g["compensated_in_order"], dtype=float), rtol=0, atol=1e-12)
+    nat = O.gptq_quantize(w, O.inverse_upper_cholesky(Hd), bits)
+    np.testing.assert_array_equal(nat["codes"][0], np.array(g["codes_natural"], dtype=int))
+    assert _act_golden_holds(golden_dir)
+
+
+@pytest.mark.parametrize("group_size", [0, 4])
+def test_act_order_with_sorted_diagonal_is_the_plain_method(group_size):
+    rng = np.random.default_rng(21)
+    d = 16
+    X = _correlated_x(64, d, rng)
+    H = O.hessian(X)
+    order = np.argsort(-np.diag(H), kind="stable")
+    H = H[np.ix_(order, order)]                     # diag(H) now descending
+    W = rng.standard_normal((10, d)) * 0.02
+    a = O.gptq_quantize_act_order(W, H, 3, group_size)
+    np.testing.assert_array_equal(a["perm"], np.arange(d))
+    p = O.gptq_quantize(W, O.inverse_upper_cholesky(O.dampen(H, 0.01)), 3, group_size)
+    np.testing.assert_array_equal(a["codes"], p["codes"])
+    np.testing.assert_array_equal(a["scales"], p["scales"])
+
+
+@pytest.mark.parametrize("group_size", [0, 8])
+def test_act_order_with_diagonal_hessian_is_rtn_in_that_order(group_size):
+    rng = np.random.default_rng(22)
+    d = 32
+    H = np.diag(rng.uniform(0.5, 5.0, d))
+    W = rng.standard_normal((12, d)) * 0.02
+    a = O.gptq_quantize_act_order(W, H, 4, group_size, block_size=8)
+    perm = np.argsort(-np.diag(H))
+    r = O.rtn_quantize(W[:, perm], 4, group_size)
+    inv = np.argsort(perm)
+    np.testing.assert_array_equal(a["codes"], r["codes"][:, inv])
+    np.testing.assert_array_equal(a["scales"], r["scales"])
+    np.testing.assert_array_equal(a["g_idx"], (inv // group_size) if group_size else np.zeros(d, dtype=int))
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("group_size", [0, 4])
+def test_act_order_equals_obs_recursion_in_that_order(seed, group_size):
+    """The explicit OBS recursion, taking the columns in act-order on the unpermuted inverse Hessian,
+    gives the same codes as the Cholesky form on the permuted problem."""
+    rng = np.random.default_rng(30 + seed)
+    d = 16
+    X = _correlated_x(64, d, rng) * rng.uniform(0.2, 3.0, d)   # distinct column scales
+    H = O.hessian(X)
+    W = rng.standard_normal((12, d)) * 0.02
+    a = O.gptq_quantize_act_order(W, H, 3, group_size)
+    o = O.obs_quantize(W, O.dampen(H, 0.01), 3, group_size, order=a["perm"])
+    np.testing.assert_array_equal(a["codes"], o["codes"])
+    np.testing.assert_allclose(a["scales"], o["scales"], rtol=1e-6)
+
+
 # ------------------------------------------------------------------------------------ mutation check
 def test_planted_mistakes_are_caught():
     """Plant plausible mistakes in what the column loop is given and check a pin fails for each."""
@@ -329,3 +404,44 @@ def test_planted_group_grid_from_original_w_is_caught(golden_dir, monkeypatch):
 
     monkeypatch.setattr(OM, "grid_params", grid_from_original)
     assert not _check_group_golden(g, Hd, w, bits, gs, 2), "group grid from the original W"
+
+
+def test_planted_act_order_mistakes_are_caught(golden_dir):
+    """Plausible mistakes in the act-order bookkeeping each fail the hand-worked act-order pin."""
+    def not_unpermuted(w, Hd, bits):
+        r = O.gptq_quantize_act_order(w, Hd, bits, damp=0.0)
+        return {**r, "codes": r["codes_in_order"]}
+
+    def ascending(w, Hd, bits):
+        return O.gptq_quantize_act_order(w, Hd, bits, damp=0.0, perm=np.argsort(np.diag(Hd), kind="stable"))
+
+    def h_not_permuted(w, Hd, bits):
+        perm = O.act_order_permutation(Hd)
+        r = O.gptq_quantize(w[:, perm], O.inverse_upper_cholesky(Hd), bits)
+        inv = np.argsort(perm)
+        return {"perm": perm, "codes": r["codes"][:, inv]}
+
+    # the OBS recursion in act-order on a layer whose permutation is not its own inverse (the golden
+    # example's [2, 1, 0] is)
+    rng = np.random.default_rng(40)
+    d = 16
+    X = _correlated_x(64, d, rng) * rng.uniform(0.2, 3.0, d)
+    H = O.hessian(X)
+    W = rng.standard_normal((12, d)) * 0.02
+    perm = O.act_order_permutation(H)
+    assert not np.array_equal(perm[perm], np.arange(d))
+    obs = O.obs_quantize(W, O.dampen(H, 0.01), 3, order=perm)["codes"]
+
+    def obs_pin_holds(fn):
+        return np.array_equal(fn(W, H, 3)["codes"], obs)
+
+    def inverse_used_as_perm_obs(W, H, bits):
+        r = O.gptq_quantize_act_order(W, H, bits)
+        return {"codes": r["codes_in_order"][:, r["perm"]]}
+
+    assert _act_golden_holds(golden_dir)
+    assert obs_pin_holds(lambda W, H, b: O.gptq_quantize_act_order(W, H, b))
+    for name, fn in {"codes left in quantization order": not_unpermuted, "ascending diag(H)": ascending,
+                     "H not permuted": h_not_permuted}.items():
+        assert not _act_golden_holds(golden_dir, fn), name
+    assert not obs_pin_holds(inverse_used_as_perm_obs), "un-permuted with perm instead of its inverse"
