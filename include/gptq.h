@@ -48,7 +48,7 @@ extern "C" {
 typedef enum {
   GPTQ_OK = 0,
   GPTQ_ERR_ARG = 1,          /* null pointer, bad size, misaligned pointer, bad combination    */
-  GPTQ_ERR_UNSUPPORTED = 2,  /* a valid option this library does not implement (act-order)    */
+  GPTQ_ERR_UNSUPPORTED = 2,  /* a valid option this library does not implement                */
   GPTQ_ERR_NOT_PD = 3,       /* device: the dampened Hessian is not positive definite          */
   GPTQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed                           */
   GPTQ_ERR_TIMEOUT = 5,      /* device: a bounded wait inside a kernel gave up                 */
@@ -58,7 +58,9 @@ typedef enum {
 typedef enum { GPTQ_BF16 = 0, GPTQ_FP16 = 1, GPTQ_FP32 = 2 } gptq_dtype;
 
 /* Flags of gptq_quant_cfg.flags. */
-#define GPTQ_FLAG_ACT_ORDER 1u /* reorder columns by descending diag(H) ("desc_act"); unsupported */
+#define GPTQ_FLAG_ACT_ORDER 1u /* columns in descending diag(H) order ("desc_act"): only with
+                                  gptq_quantize_layer_act_order, which takes the permutation; an
+                                  error (GPTQ_ERR_ARG) in gptq_quantize_layer */
 #define GPTQ_FLAG_FP32_FMA 2u  /* lazy block updates on the fp32 FMA units instead of the tensor cores
                                   (3xTF32: tf32 hi/lo splits of both operands, fp32 accumulation) */
 
@@ -167,7 +169,8 @@ GPTQ_API gptq_status gptq_prepare_uinv_static(const float* H, int64_t d, float d
  *              wait records GPTQ_ERR_TIMEOUT there (read with gptq_read_status).
  *   workspace  >= gptq_quantize_workspace_size(m, d, cfg) bytes, 256-byte aligned (holds the
  *              working copy of W in fp32 and the per-block errors).
- *   Requires d % 32 == 0 and d % block_size == 0.  flags & GPTQ_FLAG_ACT_ORDER -> UNSUPPORTED.
+ *   Requires d % 32 == 0, d % block_size == 0 and `codes` 4-byte aligned.  flags &
+ *   GPTQ_FLAG_ACT_ORDER -> GPTQ_ERR_ARG (act-order takes gptq_quantize_layer_act_order).
  *   The lazy block updates run on the tensor cores as 3xTF32 products (each operand split into a
  *   tf32 high part and a tf32 remainder, three MMAs per product, fp32 accumulation: about the
  *   accuracy of fp32 FMA); flags & GPTQ_FLAG_FP32_FMA selects fp32 FMA units instead.
@@ -177,6 +180,46 @@ GPTQ_API gptq_status gptq_quantize_layer(const void* W, int32_t w_dtype, int64_t
                                 float* scales, int32_t* zeros, int32_t* dev_status, void* workspace,
                                 size_t workspace_bytes, void* stream);
 GPTQ_API size_t gptq_quantize_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* cfg);
+
+/* ------------------------------------------------------------------------------------------
+ * Act-order ("desc_act": zhiliyouxian blog, 实践指南, off by default there; agent.csdn.net
+ * "GPTQ量化参数搜索工具", 关键参数说明).  The pages name the option without defining the order beyond
+ * "sort by activation"; here the columns are quantized in descending order of diag(H), ties by column
+ * index.  The method is unchanged on the permuted problem H -> P H P^T, W -> W P^T:
+ *   gptq_act_order(H) -> perm, H_perm;  gptq_prepare_uinv(H_perm) -> U_perm;
+ *   gptq_quantize_layer_act_order(W, U_perm, perm) -> codes in the original column order.
+ *
+ * gptq_act_order
+ *   H          [d, d] fp32, upper triangle read (as written by gptq_hessian_accumulate).
+ *   perm       int32 [d] output: perm[i] = the original column quantized at step i.
+ *   H_perm     [d, d] fp32 output: upper triangle of P H P^T, H_perm[i][j] = H[perm[i]][perm[j]]
+ *              (j >= i); strict lower triangle unspecified.  Must not alias H.  Its first d words
+ *              also serve as scratch during the call.
+ *   dev_status int32[2]: cleared at the start of the call.  NaN diagonal entries have an
+ *              unspecified place in the order.
+ *
+ * gptq_quantize_layer_act_order: gptq_quantize_layer on W P^T with U_perm, codes returned in the
+ * original column order.
+ *   W          [m, d] in the ORIGINAL column order (as for gptq_quantize_layer).
+ *   U_perm     [d, d] upper factor of the permuted dampened Hessian (gptq_prepare_uinv of H_perm).
+ *   perm       int32 [d]: a permutation of 0..d-1 (from gptq_act_order, or the caller's own order).
+ *              An entry out of range or repeated is reported on the device as {GPTQ_ERR_ARG, step}
+ *              and its columns read as zeros (no access out of bounds).
+ *   codes      [m, d] uint8 output in the original column order (4-byte aligned).
+ *   scales, zeros  [m, n_groups]: group k is steps k*group_size .. (k+1)*group_size - 1 of the
+ *              quantization order, i.e. original columns perm[k*g .. (k+1)*g - 1]; the group of
+ *              original column j is (the step at which j is quantized) / group_size.
+ *   workspace  >= gptq_quantize_act_order_workspace_size(m, d, cfg) bytes, 256-byte aligned.
+ *   cfg->flags may include GPTQ_FLAG_ACT_ORDER or not; GPTQ_FLAG_FP32_FMA applies as usual.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_act_order(const float* H, int64_t d, int32_t* perm, float* H_perm,
+                                    int32_t* dev_status, void* stream);
+GPTQ_API gptq_status gptq_quantize_layer_act_order(const void* W, int32_t w_dtype, int64_t m, int64_t d,
+                                                   const float* U_perm, const int32_t* perm,
+                                                   const gptq_quant_cfg* cfg, uint8_t* codes, float* scales,
+                                                   int32_t* zeros, int32_t* dev_status, void* workspace,
+                                                   size_t workspace_bytes, void* stream);
+GPTQ_API size_t gptq_quantize_act_order_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* cfg);
 
 /* ------------------------------------------------------------------------------------------
  * A7  Pack b-bit codes into int32 words (storage of 3-/4-bit weights for the inference kernel;

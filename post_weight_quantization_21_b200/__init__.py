@@ -9,6 +9,7 @@ the first call raises.
     U = chol((H + l*mean(diag H) I)^-1) gptq_prepare_uinv
     codes, scales, zeros              gptq_quantize_layer   (column loop + lazy block updates)
     packed int32 words                gptq_pack
+    act-order (desc_act)              gptq_act_order + gptq_quantize_layer_act_order
 
 ``LayerSolver`` strings the four calls together over preallocated buffers.
 """
@@ -23,6 +24,7 @@ __all__ = [
     "GPTQError", "lib", "gptq_hessian_accumulate", "gptq_hessian_workspace_size", "gptq_prepare_uinv",
     "gptq_prepare_workspace_size", "gptq_prepare_uinv_static", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
     "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "gptq_tensor_core_phases", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
+    "gptq_act_order", "gptq_quantize_layer_act_order", "gptq_quantize_act_order_workspace_size", "act_order_group_index",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -53,6 +55,10 @@ ABI_FUNCTIONS = {
                                    _vp, _vp, _sz, _vp]),
     "gptq_quantize_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
     "gptq_pack": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp]),
+    "gptq_act_order": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp]),
+    "gptq_quantize_layer_act_order": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, ctypes.POINTER(QuantCfg), _vp, _vp,
+                                             _vp, _vp, _vp, _sz, _vp]),
+    "gptq_quantize_act_order_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
     "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
     "gptq_status_string": (ctypes.c_char_p, [_i32]),
     "gptq_abi_version": (_i32, []),
@@ -177,6 +183,46 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, codes: torch.Tensor, s
     _check(st, "gptq_quantize_layer")
 
 
+# ------------------------------------------------------------------------------------------ act-order
+def gptq_act_order(H: torch.Tensor, perm: torch.Tensor, H_perm: torch.Tensor, status: torch.Tensor, stream=None):
+    """perm (int32 [d]) = columns by descending diag(H); H_perm (upper) = P H P^T."""
+    for t, n in ((H, "H"), (perm, "perm"), (H_perm, "H_perm"), (status, "status")):
+        _contig(t, n)
+    _check(lib().gptq_act_order(_ptr(H), H.shape[0], _ptr(perm), _ptr(H_perm), _ptr(status), _stream(stream)),
+           "gptq_act_order")
+
+
+def gptq_quantize_act_order_workspace_size(m: int, d: int, bits: int, group_size: int, block_size: int) -> int:
+    c = _cfg(bits, group_size, block_size, GPTQ_FLAG_ACT_ORDER)
+    return lib().gptq_quantize_act_order_workspace_size(m, d, ctypes.byref(c))
+
+
+def gptq_quantize_layer_act_order(W: torch.Tensor, U_perm: torch.Tensor, perm: torch.Tensor, codes: torch.Tensor,
+                                  scales: torch.Tensor, zeros: torch.Tensor, status: torch.Tensor,
+                                  workspace: torch.Tensor, bits: int, group_size: int = 0, block_size: int = 128,
+                                  flags: int = 0, stream=None):
+    """The column loop in the order ``perm`` (W in its original column order, U of the permuted Hessian);
+    codes come back in the original column order, grids per group of the quantization order."""
+    for t, n in ((W, "W"), (U_perm, "U_perm"), (perm, "perm"), (codes, "codes"), (scales, "scales"),
+                 (zeros, "zeros"), (status, "status")):
+        _contig(t, n)
+    m, d = W.shape
+    c = _cfg(bits, group_size, block_size, flags | GPTQ_FLAG_ACT_ORDER)
+    st = lib().gptq_quantize_layer_act_order(_ptr(W), _DTYPES[W.dtype], m, d, _ptr(U_perm), _ptr(perm),
+                                             ctypes.byref(c), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(status),
+                                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                             _stream(stream))
+    _check(st, "gptq_quantize_layer_act_order")
+
+
+def act_order_group_index(perm: torch.Tensor, group_size: int) -> torch.Tensor:
+    """Group of every original column under act-order: its step in ``perm`` // group_size (index
+    bookkeeping for dequantization; no arithmetic of the method)."""
+    step = torch.empty_like(perm)
+    step[perm.long()] = torch.arange(perm.numel(), dtype=perm.dtype, device=perm.device)
+    return step // group_size if group_size else torch.zeros_like(step)
+
+
 # ------------------------------------------------------------------------------------------ A7
 def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None):
     _contig(codes, "codes"), _contig(packed, "packed")
@@ -214,8 +260,10 @@ class LayerSolver:
 
 
     def __init__(self, m: int, d: int, n_tokens: int, bits: int, group_size: int = 0, block_size: int = 128,
-                 damp: float = 0.01, x_dtype=torch.bfloat16, w_dtype=torch.float16, device="cuda", flags: int = 0):
+                 damp: float = 0.01, x_dtype=torch.bfloat16, w_dtype=torch.float16, device="cuda", flags: int = 0,
+                 act_order: bool = False):
         self.m, self.d, self.n_tokens, self.flags = m, d, n_tokens, flags
+        self.act_order = act_order
         self.bits, self.group_size, self.block_size, self.damp = bits, group_size, block_size, damp
         n_groups = 1 if group_size == 0 else d // group_size
         dev = torch.device(device)
@@ -229,12 +277,17 @@ class LayerSolver:
         self.zeros = torch.empty(m, n_groups, dtype=torch.int32, device=dev)
         self.packed = torch.empty(m, d * bits // 32, dtype=torch.int32, device=dev)
         # one device status word per call (prepare and quantize clear theirs when they start)
-        self.status = torch.zeros(3, 2, dtype=torch.int32, device=dev)  # rows: hessian, prepare, quantize
+        # rows: hessian, prepare, quantize, act-order permutation
+        self.status = torch.zeros(4, 2, dtype=torch.int32, device=dev)
         self.host_chunk = min(n_tokens, self.HOST_CHUNK_TOKENS)
+        q_ws = (gptq_quantize_act_order_workspace_size(m, d, bits, group_size, block_size) if act_order
+                else gptq_quantize_workspace_size(m, d, bits, group_size, block_size))
+        if act_order:
+            self.perm = torch.empty(d, dtype=torch.int32, device=dev)
+            self.H_perm = torch.empty(d, d, dtype=torch.float32, device=dev)
         ws = max(gptq_hessian_workspace_size(n_tokens, d, x_dtype),
                  gptq_hessian_workspace_size(self.host_chunk, d, x_dtype) if self.host_chunk else 0,
-                 gptq_prepare_workspace_size(d), gptq_quantize_workspace_size(m, d, bits, group_size, block_size),
-                 256)
+                 gptq_prepare_workspace_size(d), q_ws, 256)
         self.workspace = torch.empty(ws, dtype=u8, device=dev)
         self._copy_stream = None
 
@@ -242,11 +295,21 @@ class LayerSolver:
         gptq_hessian_accumulate(self.X, self.H, self.status[0], self.workspace, 2.0, False, stream)
 
     def prepare(self, stream=None):
-        gptq_prepare_uinv(self.H, self.U, self.status[1], self.workspace, self.damp, stream)
+        """U of the dampened Hessian; with act-order, the permutation first and U of P H P^T."""
+        if self.act_order:
+            gptq_act_order(self.H, self.perm, self.H_perm, self.status[3], stream)
+            gptq_prepare_uinv(self.H_perm, self.U, self.status[1], self.workspace, self.damp, stream)
+        else:
+            gptq_prepare_uinv(self.H, self.U, self.status[1], self.workspace, self.damp, stream)
 
     def quantize(self, stream=None):
-        gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.status[2], self.workspace,
-                            self.bits, self.group_size, self.block_size, self.flags, stream)
+        if self.act_order:
+            gptq_quantize_layer_act_order(self.W, self.U, self.perm, self.codes, self.scales, self.zeros,
+                                          self.status[2], self.workspace, self.bits, self.group_size,
+                                          self.block_size, self.flags, stream)
+        else:
+            gptq_quantize_layer(self.W, self.U, self.codes, self.scales, self.zeros, self.status[2], self.workspace,
+                                self.bits, self.group_size, self.block_size, self.flags, stream)
 
     def pack(self, stream=None):
         gptq_pack(self.codes, self.bits, self.packed, stream)

@@ -20,11 +20,13 @@ size_t dtype_size(int32_t t) { return t == GPTQ_FP32 ? 4 : 2; }
 
 constexpr int64_t kMaxDim = 1 << 20;  // channel / row limit (keeps every 32-bit tile index in range)
 
-gptq_status check_cfg(const gptq_quant_cfg* cfg, int64_t d) {
+// act_order: whether the caller takes the act-order path (GPTQ_FLAG_ACT_ORDER allowed); the plain
+// gptq_quantize_layer has no permutation argument, so the flag is an error there
+gptq_status check_cfg(const gptq_quant_cfg* cfg, int64_t d, bool act_order = false) {
   if (cfg == nullptr) return GPTQ_ERR_ARG;
   if (cfg->bits < 2 || cfg->bits > 4) return GPTQ_ERR_ARG;
   if (cfg->block_size != 32 && cfg->block_size != 64 && cfg->block_size != 128) return GPTQ_ERR_ARG;
-  if (cfg->flags & GPTQ_FLAG_ACT_ORDER) return GPTQ_ERR_UNSUPPORTED;
+  if ((cfg->flags & GPTQ_FLAG_ACT_ORDER) && !act_order) return GPTQ_ERR_ARG;
   if (cfg->flags & ~(GPTQ_FLAG_ACT_ORDER | GPTQ_FLAG_FP32_FMA)) return GPTQ_ERR_ARG;
   if (d % cfg->block_size) return GPTQ_ERR_ARG;
   const int g = cfg->group_size;
@@ -45,7 +47,7 @@ int32_t gptq_abi_version(void) { return GPTQ_ABI_VERSION; }
 uint64_t gptq_kernel_launches(void) { return gptq::g_launches.load(std::memory_order_relaxed); }
 
 int32_t gptq_tensor_core_phases(int64_t m, int64_t d, int64_t n_tokens, int32_t x_dtype, const gptq_quant_cfg* cfg) {
-  if (m <= 0 || d <= 0 || n_tokens < 0 || d > kMaxDim || !valid_dtype(x_dtype) || check_cfg(cfg, d) != GPTQ_OK)
+  if (m <= 0 || d <= 0 || n_tokens < 0 || d > kMaxDim || !valid_dtype(x_dtype) || check_cfg(cfg, d, true) != GPTQ_OK)
     return -1;
   int32_t mask = 0;
   if (gptq::hessian_tc_supported(n_tokens, d, x_dtype)) mask |= GPTQ_TC_HESSIAN;
@@ -130,13 +132,46 @@ gptq_status gptq_quantize_layer(const void* W, int32_t w_dtype, int64_t m, int64
   gptq_status st = check_cfg(cfg, d);
   if (st != GPTQ_OK) return st;
   if (!W || !U || !codes || !scales || !zeros || !dev_status) return GPTQ_ERR_ARG;
-  if (!aligned(W, dtype_size(w_dtype)) || !aligned(U, 16) || !aligned(scales, 4) || !aligned(zeros, 4) ||
-      !aligned(dev_status, 4))
+  if (!aligned(W, dtype_size(w_dtype)) || !aligned(U, 16) || !aligned(codes, 4) || !aligned(scales, 4) ||
+      !aligned(zeros, 4) || !aligned(dev_status, 4))
     return GPTQ_ERR_ARG;
   const size_t need = gptq::quantize_workspace(m, d, cfg->block_size);
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return GPTQ_ERR_WORKSPACE;
   return gptq::quantize_launch(W, w_dtype, m, d, U, *cfg, codes, scales, zeros, dev_status, workspace,
                                static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptq_act_order(const float* H, int64_t d, int32_t* perm, float* H_perm, int32_t* dev_status,
+                           void* stream) {
+  if (d <= 0 || d > kMaxDim || H == nullptr || perm == nullptr || H_perm == nullptr || dev_status == nullptr)
+    return GPTQ_ERR_ARG;
+  if (!aligned(H, 4) || !aligned(perm, 4) || !aligned(H_perm, 4) || !aligned(dev_status, 4)) return GPTQ_ERR_ARG;
+  if ((const void*)H == (const void*)H_perm) return GPTQ_ERR_ARG;
+  return gptq::act_order_launch(H, d, perm, H_perm, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+size_t gptq_quantize_act_order_workspace_size(int64_t m, int64_t d, const gptq_quant_cfg* cfg) {
+  if (m <= 0 || d <= 0 || d > kMaxDim || m > kMaxDim * 64 || cfg == nullptr) return 0;
+  if (check_cfg(cfg, d, true) != GPTQ_OK) return 0;
+  return gptq::quantize_act_order_workspace(m, d, cfg->block_size);
+}
+
+gptq_status gptq_quantize_layer_act_order(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U_perm,
+                                          const int32_t* perm, const gptq_quant_cfg* cfg, uint8_t* codes,
+                                          float* scales, int32_t* zeros, int32_t* dev_status, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(w_dtype) || m <= 0 || d <= 0 || d > kMaxDim || m > kMaxDim * 64 || d % 32)
+    return GPTQ_ERR_ARG;
+  gptq_status st = check_cfg(cfg, d, true);
+  if (st != GPTQ_OK) return st;
+  if (!W || !U_perm || !perm || !codes || !scales || !zeros || !dev_status) return GPTQ_ERR_ARG;
+  if (!aligned(W, dtype_size(w_dtype)) || !aligned(U_perm, 16) || !aligned(perm, 4) || !aligned(codes, 4) ||
+      !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(dev_status, 4))
+    return GPTQ_ERR_ARG;
+  const size_t need = gptq::quantize_act_order_workspace(m, d, cfg->block_size);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return GPTQ_ERR_WORKSPACE;
+  return gptq::quantize_act_order_launch(W, w_dtype, m, d, U_perm, perm, *cfg, codes, scales, zeros, dev_status,
+                                         workspace, static_cast<cudaStream_t>(stream));
 }
 
 gptq_status gptq_pack(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed, void* stream) {

@@ -64,9 +64,19 @@ bool quantize_fused(int64_t m, int64_t d);  // one launch per layer (U resident 
 // the lazy block updates run as 3xTF32 tensor-core products (the per-block path without GPTQ_FLAG_FP32_FMA,
 // with a tile count that fits 32 bits); the launch takes exactly this path or fails
 bool quantize_lazy_on_tensor_cores(int64_t m, int64_t d, uint32_t flags);
+// clear_status = false keeps what earlier launches of the same call recorded in the status word
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
-                            int32_t* status, void* workspace, cudaStream_t stream);
+                            int32_t* status, void* workspace, cudaStream_t stream, bool clear_status = true);
+
+// act-order (act_order.cu)
+gptq_status act_order_launch(const float* H, int64_t d, int32_t* perm, float* H_perm, int32_t* status,
+                             cudaStream_t stream);
+size_t quantize_act_order_workspace(int64_t m, int64_t d, int block_size);
+gptq_status quantize_act_order_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d, const float* U_perm,
+                                      const int32_t* perm, const gptq_quant_cfg& cfg, uint8_t* codes,
+                                      float* scales, int32_t* zeros, int32_t* status, void* workspace,
+                                      cudaStream_t stream);
 
 // A7
 gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,

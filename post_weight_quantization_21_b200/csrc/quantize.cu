@@ -675,9 +675,9 @@ bool quantize_lazy_on_tensor_cores(int64_t m, int64_t d, uint32_t flags) {
 
 gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d64, const float* U,
                             const gptq_quant_cfg& cfg, uint8_t* codes, float* scales, int32_t* zeros,
-                            int32_t* status, void* workspace, cudaStream_t s) {
+                            int32_t* status, void* workspace, cudaStream_t s, bool clear_status) {
   const int d = (int)d64;
-  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), s));
+  if (clear_status) GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), s));
   char* ws = static_cast<char*>(workspace);
   float* ww = reinterpret_cast<float*>(ws);
   float* err = reinterpret_cast<float*>(ws + align_up((size_t)m * d * sizeof(float), 256));

@@ -55,6 +55,10 @@ def test_workspace_sizes(lib):
     assert lib.gptq_prepare_workspace_size(0) == 0
 
 
+def other_ptr():
+    return ctypes.c_void_p(8192)
+
+
 def test_validation_rejects_bad_arguments_without_a_device(lib):
     cfg = g.QuantCfg(4, 0, 128, 0)
     fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
@@ -65,7 +69,20 @@ def test_validation_rejects_bad_arguments_without_a_device(lib):
     assert st == g.GPTQ_ERR_ARG                               # bits = 5
     act = g.QuantCfg(4, 0, 128, g.GPTQ_FLAG_ACT_ORDER)
     st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(act), fake, fake, fake, fake, fake, 1 << 20, None)
-    assert st == g.GPTQ_ERR_UNSUPPORTED
+    assert st == g.GPTQ_ERR_ARG                               # act-order needs the permutation argument
+    assert lib.gptq_quantize_act_order_workspace_size(8, 128, ctypes.byref(act)) > \
+        lib.gptq_quantize_workspace_size(8, 128, ctypes.byref(cfg))
+    st = lib.gptq_quantize_layer_act_order(fake, 1, 8, 128, fake, None, ctypes.byref(act), fake, fake, fake, fake,
+                                           fake, 1 << 24, None)
+    assert st == g.GPTQ_ERR_ARG                               # no permutation
+    st = lib.gptq_quantize_layer_act_order(fake, 1, 8, 128, fake, fake, ctypes.byref(act), fake, fake, fake, fake,
+                                           fake, 16, None)
+    assert st == g.GPTQ_ERR_WORKSPACE
+    odd = ctypes.c_void_p(257)
+    st = lib.gptq_quantize_layer(fake, 1, 8, 128, fake, ctypes.byref(cfg), odd, fake, fake, fake, fake, 1 << 20, None)
+    assert st == g.GPTQ_ERR_ARG                               # codes not 4-byte aligned
+    assert lib.gptq_act_order(fake, 16, fake, fake, fake, None) == g.GPTQ_ERR_ARG      # H_perm aliases H
+    assert lib.gptq_act_order(fake, 0, fake, other_ptr(), fake, None) == g.GPTQ_ERR_ARG
     grp = g.QuantCfg(4, 96, 128, 0)                           # 96 and 128 do not divide one another
     st = lib.gptq_quantize_layer(fake, 1, 8, 384, fake, ctypes.byref(grp), fake, fake, fake, fake, fake, 1 << 20, None)
     assert st == g.GPTQ_ERR_ARG
