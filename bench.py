@@ -39,6 +39,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--layer", default=DEFAULT_LAYER)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--mode", default="layers", choices=["layers", "sharded"],
+                   help="N > 1: 'layers' = each rank solves its own layer (weak scaling); 'sharded' = one layer "
+                        "split across the ranks (tokens for H + all-reduce, rows for the solve; strong scaling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=None,
                    help="end-to-end steps (default: 10, or 3 on layers whose step takes over 0.5 s)")
@@ -65,6 +68,43 @@ def layer_for_rank(L, rank: int):
     data-path collective."""
     import dataclasses
     return dataclasses.replace(L, seed=L.seed + rank)
+
+
+class ShardedRunner:
+    """One layer split across the ranks (ShardedLayerSolver) behind the calls the timing loop makes."""
+
+    def __init__(self, L, dev):
+        from post_weight_quantization_21_b200.sharded import ShardedLayerSolver
+        from post_weight_quantization_21_b200 import workloads as wl
+        self.s = ShardedLayerSolver(L.m, L.d, L.n_tokens, L.bits, L.group_size, L.block_size, L.damp, L.x_dtype,
+                                    L.w_dtype, dev, token_align=wl.CHUNK_TOKENS)
+        self.W, self.X = self.s.W_local, self.s.X_local
+        (t0, t1), (r0, r1) = self.s.tokens, self.s.rows
+        self.n_local, self.m_local = t1 - t0, r1 - r0
+        for c in range(t0 // wl.CHUNK_TOKENS, (t1 + wl.CHUNK_TOKENS - 1) // wl.CHUNK_TOKENS):
+            chunk = wl.make_x_chunk(L, c, dev)
+            a = c * wl.CHUNK_TOKENS - t0
+            self.X[a:a + chunk.shape[0]].copy_(chunk)
+        self.W.copy_(wl.make_w(L, device=dev)[r0:r1])
+        self.packed, self.scales, self.zeros = self.s.packed, self.s.scales, self.s.zeros
+
+    def hessian(self, stream):
+        self.s.hessian()
+
+    def prepare(self, stream):
+        self.s.prepare()
+
+    def quantize(self, stream):
+        self.s.quantize()
+
+    def pack(self, stream):
+        self.s.pack()
+
+    def check_status(self, stream):
+        self.s.check_status()
+
+    def run_host(self, W_h, X_h, out_p, out_s, out_z, stream):
+        self.s.run_host(W_h, X_h, out_p, out_s, out_z)
 
 
 def peaks():
@@ -331,11 +371,17 @@ def main():
     dev = torch.device("cuda", local)
     pk = peaks()
 
-    solver = g.LayerSolver(L.m, L.d, L.n_tokens, L.bits, L.group_size, L.block_size, L.damp, L.x_dtype,
-                           L.w_dtype, device=dev)
     # seeded inputs made on the device (the large layers' X is tens of GB); host copies below
-    solver.W.copy_(wl.make_w(L, device=dev))
-    wl.make_x(L, device=dev, out=solver.X)
+    if args.mode == "sharded":
+        L = wl.LAYERS[args.layer]                     # one layer shared by all ranks
+        solver = ShardedRunner(L, dev)
+        n_eff, m_eff, job_weights = solver.n_local, solver.m_local, L.m * L.d
+    else:
+        solver = g.LayerSolver(L.m, L.d, L.n_tokens, L.bits, L.group_size, L.block_size, L.damp, L.x_dtype,
+                               L.w_dtype, device=dev)
+        solver.W.copy_(wl.make_w(L, device=dev))
+        wl.make_x(L, device=dev, out=solver.X)
+        n_eff, m_eff, job_weights = L.n_tokens, L.m, world * L.m * L.d
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -382,7 +428,7 @@ def main():
     phase_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
     total_ms = slowest_rank_ms(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = world * L.m * L.d / (ms_per_step * 1e-3)
+    value = job_weights / (ms_per_step * 1e-3)
 
     # end to end through the host: pinned inputs in, packed codes + grids out, every step
     W_h = torch.empty(solver.W.shape, dtype=solver.W.dtype, pin_memory=True)
@@ -390,9 +436,9 @@ def main():
     W_h.copy_(solver.W)
     X_h.copy_(solver.X)
     n_groups = 1 if L.group_size == 0 else L.d // L.group_size
-    out_p = torch.empty(L.m, L.d * L.bits // 32, dtype=torch.int32, pin_memory=True)
-    out_s = torch.empty(L.m, n_groups, dtype=torch.float32, pin_memory=True)
-    out_z = torch.empty(L.m, n_groups, dtype=torch.int32, pin_memory=True)
+    out_p = torch.empty(m_eff, L.d * L.bits // 32, dtype=torch.int32, pin_memory=True)
+    out_s = torch.empty(m_eff, n_groups, dtype=torch.float32, pin_memory=True)
+    out_z = torch.empty(m_eff, n_groups, dtype=torch.int32, pin_memory=True)
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else (3 if ms_per_step > 500.0 else 10)
     solver.run_host(W_h, X_h, out_p, out_s, out_z, stream)
     torch.cuda.synchronize(dev)
@@ -418,10 +464,11 @@ def main():
     fp32_peak = fp32_meas
     tf32x3_peak = bf16_peak * TF32_PER_BF16 / 3.0   # three tf32 MMAs per fp32-accurate product
     tc = g.gptq_tensor_core_phases(L.m, L.d, L.n_tokens, L.x_dtype, L.bits, L.group_size, L.block_size)
-    h_flops = L.n_tokens * L.d * (L.d + 1)                 # symmetric half of 2 N d^2
+    # this rank's algorithmic work (sharded mode: its tokens and rows; the prepare step is replicated)
+    h_flops = n_eff * L.d * (L.d + 1)                      # symmetric half of 2 N d^2
     p_flops = 2.0 / 3.0 * L.d ** 3                          # Cholesky + triangular inverse
-    q_flops = float(L.m) * L.d * L.d                        # column loop + lazy updates
-    k_bytes = L.m * L.d * (1 + L.bits / 8)                  # pack: codes in, words out
+    q_flops = float(m_eff) * L.d * L.d                      # column loop + lazy updates
+    k_bytes = m_eff * L.d * (1 + L.bits / 8)                # pack: codes in, words out
     p_peak, p_pipe = (tf32x3_peak, "tensor(3xtf32)") if tc & g.GPTQ_TC_PREPARE else (fp32_peak, "fp32 FMA")
     q_peak, q_pipe = (tf32x3_peak, "tensor(3xtf32)") if tc & g.GPTQ_TC_LAZY else (fp32_peak, "fp32 FMA")
     bf16_src = f"{pk['source']} bf16 {'sustained' if long_region else 'burst'}"
@@ -449,7 +496,7 @@ def main():
     roof_hessian = {"bound": "tensor", "kernel": "hessian_tc_kernel (A1, one launch per step)",
                     "achieved": h_tflops, "peak": bf16_peak, "unit": "TFLOP/s", "frac": h_tflops / bf16_peak,
                     "peak_source": bf16_src,
-                    "algorithmic": f"N*d*(d+1) = {h_flops:.4g} flop per launch (N={L.n_tokens}, d={L.d})",
+                    "algorithmic": f"N*d*(d+1) = {h_flops:.4g} flop per launch (N={n_eff}, d={L.d})",
                     "traffic": kernel_traffic("hessian_" + L.name, hessian_sources())}
     # the phase that takes the largest share of the step
     work = {"hessian": (h_flops, "N*d*(d+1) flop"), "prepare": (p_flops, "2/3 d^3 flop"),
@@ -473,10 +520,14 @@ def main():
                     "algorithmic": f"{work[top][1]} = {work[top][0]:.4g} per step (one phase = one unit)",
                     "traffic": None}
 
+    cfg = config_of(L)
+    cfg["parallelism"] = (f"{world} ranks, one layer: tokens sharded for H + all-reduce, U replicated, rows "
+                          "sharded" if args.mode == "sharded" else f"{world} independent layer(s), one per rank")
     line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(L),
-            "e2e": {"value": world * L.m * L.d / (e2e_ms * 1e-3), "unit": "weights/s", "ms_per_step": e2e_ms,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if args.mode == "sharded" else "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+            "e2e": {"value": job_weights / (e2e_ms * 1e-3), "unit": "weights/s", "ms_per_step": e2e_ms,
                     "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches), "roofline": roofline, "roofline_hessian": roof_hessian,
             "phases": phases, "phase_roofline_ms": roof_ms, "end_to_end_roofline_frac": roof_ms / ms_per_step,
