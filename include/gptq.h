@@ -261,6 +261,15 @@ GPTQ_API uint64_t gptq_kernel_launches(void);
 GPTQ_API int32_t gptq_tensor_core_phases(int64_t m, int64_t d, int64_t n_tokens, int32_t x_dtype,
                                          const gptq_quant_cfg* cfg);
 
+/* Failure-detection test hook (no counterpart on the pages).  Makes the NEXT Hessian launch on the
+ * tensor-core path (16-bit X, see GPTQ_TC_HESSIAN) exercise its timeout path without any fault: its
+ * MMA-issuing thread first waits, for at most `cycles` clock cycles, on a barrier that nothing arrives
+ * on, gives up, records {GPTQ_ERR_TIMEOUT, 5} in that call's status word and raises the kernel's abort
+ * flag; the other roles leave, the copies already issued land (their waits keep the full bound), TMEM
+ * is freed and the kernel returns.  H is then unspecified.  The request is taken by one launch (any
+ * thread's); cycles <= 0 cancels it.  Calls made afterwards run normally. */
+GPTQ_API void gptq_test_hessian_timeout(int64_t cycles);
+
 #ifdef __cplusplus
 }
 #endif

@@ -59,6 +59,7 @@ ABI_FUNCTIONS = {
     "gptq_quantize_layer_act_order": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, ctypes.POINTER(QuantCfg), _vp, _vp,
                                              _vp, _vp, _vp, _sz, _vp]),
     "gptq_quantize_act_order_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
+    "gptq_test_hessian_timeout": (None, [_i64]),
     "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
     "gptq_status_string": (ctypes.c_char_p, [_i32]),
     "gptq_abi_version": (_i32, []),

@@ -17,6 +17,8 @@
 //               partial) to global memory.
 // Every mbarrier wait is bounded: on a timeout the kernel records GPTQ_ERR_TIMEOUT, lets the
 // other roles leave, waits (bounded) for its own TMA copies and MMAs in flight, frees TMEM, returns.
+#include <atomic>
+
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -85,6 +87,7 @@ struct TcArgs {
   float* H;
   float* partial;
   int32_t* status;
+  long long test_wait;  // > 0: the failure-detection test (see gptq_test_hessian_timeout)
 };
 
 using namespace tc;
@@ -193,6 +196,9 @@ __global__ void __launch_bounds__(THREADS, 1) hessian_tc_kernel(const __grid_con
       uint32_t stage = 0, chunk = 0;
       bool ok = true;
       const uint32_t smem0 = smem_u32(smem);
+      // failure-detection test only: wait, for at most test_wait cycles, on a barrier nothing arrives
+      // on before this thread's own final commit, so the wait gives up and the timeout path runs
+      if (a.test_wait > 0) ok = mbar_wait(drain, 0, abort_flag, a.status, 5, a.test_wait);
       for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
         int bi, bj, s;
         unit_coords(u, a, bi, bj, s);
@@ -346,6 +352,9 @@ __global__ void hessian_tc_reduce_kernel(const float* __restrict__ partial, int 
 
 constexpr int kSmemBytes = STAGES * STAGE_BYTES + 1024 + 256;
 
+// One-shot request of the failure-detection test (gptq_test_hessian_timeout), taken by the next launch.
+std::atomic<long long> g_test_wait{0};
+
 }  // namespace
 
 bool hessian_tc_supported(int64_t n_tokens, int64_t d, int32_t x_dtype) {
@@ -398,6 +407,7 @@ gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, 
   a.H = H;
   a.partial = static_cast<float*>(workspace);
   a.status = status;
+  a.test_wait = g_test_wait.exchange(0);
   const int grid = p.units < sms ? p.units : sms;
   hessian_tc_kernel<<<grid, THREADS, kSmemBytes, stream>>>(map, a);
   GPTQ_LAUNCH_CHECK();
@@ -410,3 +420,5 @@ gptq_status hessian_tc_launch(const void* X, int32_t x_dtype, int64_t n_tokens, 
 }
 
 }  // namespace gptq
+
+extern "C" void gptq_test_hessian_timeout(int64_t cycles) { gptq::g_test_wait.store(cycles > 0 ? cycles : 0); }

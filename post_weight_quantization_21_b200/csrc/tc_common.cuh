@@ -43,16 +43,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity.  Gives up (returns false) when another role has
-// aborted, or after kWaitCycles, in which case it raises the abort flag and records a timeout.
+// aborted, or after `limit` cycles, in which case it raises the abort flag and records a timeout.
 __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
-                                 int where) {
+                                 int where, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         report_status(status, GPTQ_ERR_TIMEOUT, where);
         return false;

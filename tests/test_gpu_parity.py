@@ -66,6 +66,26 @@ def test_hessian_tensor_core_accumulate_mode():
     assert S.upper_rel_fro(H.cpu().numpy(), Href) <= S.H_REL_FRO
 
 
+def test_hessian_timeout_is_reported_and_the_context_stays_usable():
+    """Failure detection without a fault: the test hook makes the tensor-core Hessian's MMA issuer give
+    up a bounded wait (about 0.5 ms at the base clock) on a barrier nothing arrives on.  The call's
+    status word reports GPTQ_ERR_TIMEOUT at wait 5; the next call on the same stream runs normally."""
+    X = _x(8192, 512, torch.bfloat16, seed=17).to(S.dev())
+    n, d = X.shape
+    assert g.gptq_tensor_core_phases(64, d, n, X.dtype, 4) & g.GPTQ_TC_HESSIAN
+    H = torch.empty(d, d, device=S.dev())
+    ws = torch.empty(max(g.gptq_hessian_workspace_size(n, d, X.dtype), 256), dtype=torch.uint8, device=S.dev())
+    st = torch.zeros(2, dtype=torch.int32, device=S.dev())
+    g.lib().gptq_test_hessian_timeout(1_000_000)
+    g.gptq_hessian_accumulate(X, H, st, ws, 2.0, False)
+    code, detail = g.gptq_read_status(st)
+    assert (code, detail) == (g.GPTQ_ERR_TIMEOUT, 5)
+    g.gptq_hessian_accumulate(X, H, st, ws, 2.0, False)      # a fresh sum clears the status word
+    code, detail = g.gptq_read_status(st)
+    assert code == g.GPTQ_OK, (code, detail)
+    assert S.upper_rel_fro(H.cpu().numpy(), oracle.hessian(X.cpu().double().numpy())) <= S.H_REL_FRO
+
+
 def test_hessian_full_size_opt125m_layer():
     L = wl.LAYERS["opt125m_768x768"]
     X = wl.make_x(L)
