@@ -233,6 +233,29 @@ GPTQ_API gptq_status gptq_pack(const uint8_t* codes, int64_t m, int64_t d, int32
                       void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Inference with the packed weights: Y = X @ What^T with What[r, j] = scale[r, g(j)] * (q[r, j] -
+ * zero[r, g(j)]), g(j) = j / group_size (0 per-row), q read from the packed words (FDE breakdown,
+ * section 01, last paragraph: kernels that read the 3-bit weights and dequantize them on the fly).
+ * For a few input rows (batch): every packed word is read once from HBM.
+ *
+ *   packed     [m, d*bits/32] int32 from gptq_pack; scales / zeros [m, n_groups] from
+ *              gptq_quantize_layer.  Under act-order the groups follow the quantization order: pass
+ *              the codes in that order (codes[:, perm] packed) and X with its columns permuted alike.
+ *   X          [batch, d] row-major, BF16 / FP16 / FP32, 16-byte aligned.  1 <= batch <= 1024
+ *              (processed four rows at a time).
+ *   Y          [batch, m] fp32 output.
+ *   workspace  >= gptq_dequant_matmul_workspace_size(m, d, batch) bytes, 256-byte aligned (partial
+ *              sums of the column tiles; the final sum runs in tile order, so results are
+ *              deterministic).
+ *   Requires d % 32 == 0, bits in {2, 3, 4}, group_size 0 or a multiple of 32 dividing d.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_dequant_matmul(const int32_t* packed, const float* scales, const int32_t* zeros,
+                                         int64_t m, int64_t d, int32_t bits, int32_t group_size, const void* X,
+                                         int32_t x_dtype, int64_t batch, float* Y, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+GPTQ_API size_t gptq_dequant_matmul_workspace_size(int64_t m, int64_t d, int64_t batch);
+
+/* ------------------------------------------------------------------------------------------
  * Status helpers.
  * gptq_read_status: synchronizes `stream`, copies the device status word to the host, returns the
  * code it holds (GPTQ_OK if clear) and stores its detail (e.g. the failing pivot) in *detail when

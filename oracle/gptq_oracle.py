@@ -46,7 +46,7 @@ __all__ = [
     "inverse_upper_cholesky_reversed", "grid_params", "quantize_codes", "dequantize",
     "gptq_quantize", "rtn_quantize", "obs_quantize", "conditional_ls_values",
     "bruteforce_best_codes", "reconstruction_error", "pack_codes", "unpack_codes", "gptq_layer",
-    "act_order_permutation", "gptq_quantize_act_order", "act_order_group_index",
+    "act_order_permutation", "gptq_quantize_act_order", "act_order_group_index", "dequant_matmul",
 ]
 
 
@@ -372,6 +372,23 @@ def gptq_quantize_act_order(W, H, bits: int, group_size: int = 0, block_size: in
     return {"codes": r["codes"][:, inv], "Wq": r["Wq"][:, inv], "scales": r["scales"], "zeros": r["zeros"],
             "perm": perm, "g_idx": act_order_group_index(perm, group_size), "U": U,
             "codes_in_order": r["codes"]}
+
+
+# --------------------------------------------------------------------------------------------
+# Inference with the packed weights.  [FDE] section 01, last paragraph: custom kernels read the 3-bit
+# weights and dequantize them on the fly (the 3.25x generation speed-up on A100).  What that kernel
+# computes is the layer's product with the dequantized weights: Y = X_in @ What^T with
+# What[r, j] = scale[r, g(j)] * (q[r, j] - zero[r, g(j)]), g(j) = j // group_size (0 per-row), the codes
+# read from the packed words (A7 layout).  X_in [batch, d] -> Y [batch, m].
+# --------------------------------------------------------------------------------------------
+def dequant_matmul(packed, scales, zeros, bits: int, group_size: int, d: int, X_in) -> np.ndarray:
+    codes = unpack_codes(packed, bits, d)
+    m = codes.shape[0]
+    gs = d if group_size == 0 else group_size
+    s = np.repeat(np.asarray(scales, dtype=np.float64).reshape(m, -1), gs, axis=1)
+    z = np.repeat(np.asarray(zeros, dtype=np.float64).reshape(m, -1), gs, axis=1)
+    What = dequantize(codes, s, z)
+    return np.asarray(X_in, dtype=np.float64) @ What.T
 
 
 # --------------------------------------------------------------------------------------------

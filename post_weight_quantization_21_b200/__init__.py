@@ -25,6 +25,7 @@ __all__ = [
     "gptq_prepare_workspace_size", "gptq_prepare_uinv_static", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
     "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "gptq_tensor_core_phases", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
     "gptq_act_order", "gptq_quantize_layer_act_order", "gptq_quantize_act_order_workspace_size", "act_order_group_index",
+    "gptq_dequant_matmul", "gptq_dequant_matmul_workspace_size",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -60,6 +61,8 @@ ABI_FUNCTIONS = {
                                              _vp, _vp, _vp, _sz, _vp]),
     "gptq_quantize_act_order_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
     "gptq_test_hessian_timeout": (None, [_i64]),
+    "gptq_dequant_matmul": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _i32, _i64, _vp, _vp, _sz, _vp]),
+    "gptq_dequant_matmul_workspace_size": (_sz, [_i64, _i64, _i64]),
     "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
     "gptq_status_string": (ctypes.c_char_p, [_i32]),
     "gptq_abi_version": (_i32, []),
@@ -229,6 +232,24 @@ def gptq_pack(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None)
     _contig(codes, "codes"), _contig(packed, "packed")
     m, d = codes.shape
     _check(lib().gptq_pack(_ptr(codes), m, d, bits, _ptr(packed), _stream(stream)), "gptq_pack")
+
+
+# ------------------------------------------------------------------------------------------ inference
+def gptq_dequant_matmul_workspace_size(m: int, d: int, batch: int) -> int:
+    return lib().gptq_dequant_matmul_workspace_size(m, d, batch)
+
+
+def gptq_dequant_matmul(packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int, group_size: int,
+                        X: torch.Tensor, Y: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """Y [batch, m] (fp32) = X [batch, d] @ What^T, What dequantized on the fly from the packed codes."""
+    for t, n in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (X, "X"), (Y, "Y")):
+        _contig(t, n)
+    m = packed.shape[0]
+    batch, d = X.shape
+    st = lib().gptq_dequant_matmul(_ptr(packed), _ptr(scales), _ptr(zeros), m, d, bits, group_size, _ptr(X),
+                                   _DTYPES[X.dtype], batch, _ptr(Y), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "gptq_dequant_matmul")
 
 
 def gptq_tensor_core_phases(m: int, d: int, n_tokens: int, x_dtype, bits: int, group_size: int = 0,

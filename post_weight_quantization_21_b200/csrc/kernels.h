@@ -78,6 +78,12 @@ gptq_status quantize_act_order_launch(const void* W, int32_t w_dtype, int64_t m,
                                       float* scales, int32_t* zeros, int32_t* status, void* workspace,
                                       cudaStream_t stream);
 
+// inference with the packed weights (dequant_matmul.cu)
+size_t dequant_matmul_workspace(int64_t m, int64_t d, int64_t batch);
+gptq_status dequant_matmul_launch(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m,
+                                  int64_t d, int32_t bits, int32_t group_size, const void* X, int32_t x_dtype,
+                                  int64_t batch, float* Y, void* workspace, cudaStream_t stream);
+
 // A7
 gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,
                         cudaStream_t stream);

@@ -40,6 +40,11 @@ def pytest_terminal_summary(terminalreporter):
     """Code mismatches of every GPU parity comparison with the oracle (near-tie decisions and the
     trajectories that follow them), one line per comparison."""
     sup = sys.modules.get("gpu_support")
+    notes = getattr(sup, "NOTES", None)
+    if notes:
+        terminalreporter.section("measured figures")
+        for label, text in notes:
+            terminalreporter.write_line(f"{label}: {text}")
     log = getattr(sup, "PARITY_LOG", None)
     if not log:
         return

@@ -15,6 +15,8 @@ E_REL = 0.02             # layer reconstruction error, relative
 
 # every compare_quantization call appends (label, stats) here; the session summary prints them
 PARITY_LOG: list[tuple[str, dict]] = []
+# other measured figures a test wants in the session summary (label, text)
+NOTES: list[tuple[str, str]] = []
 
 
 def dev():

@@ -155,8 +155,8 @@ def test_prepare_widest_layer_sampled_rows_and_columns():
     R = HV[:, nr:]
     R[cols, np.arange(len(cols))] -= 1.0
     c_err = np.linalg.norm(R, axis=0).max()
-    print(WIDEST, "sampled rows: max |U Hd U^T - I|", g_err, "; sampled columns: max ||Hd U^T U e_j - e_j||",
-          c_err)
+    S.NOTES.append((WIDEST + " U", f"sampled rows max |U Hd U^T - I| = {g_err:.3e} (bound {L.d * 6e-8:.3e}); "
+                                   f"sampled columns max ||Hd U^T U e_j - e_j|| = {c_err:.3e}"))
     # fp32 factorisation and inversion of a d x d matrix: the identity's entries carry sums of d
     # rounded products each; d * eps32 bounds their linear growth
     assert g_err <= L.d * 6e-8, g_err
@@ -231,7 +231,7 @@ def test_end_to_end_chained_layer(name, n_tokens):
     rel = np.linalg.norm(Ug - U) / np.linalg.norm(U)
     ev = np.linalg.eigvalsh(Hd)
     kappa = ev[-1] / ev[0]
-    print(name, "U rel err", rel, "kappa", kappa)
+    S.NOTES.append((f"{name} chained U", f"rel err {rel:.3e}, kappa {kappa:.3e}"))
     assert rel <= max(1e-5, 10 * kappa * 6e-8), (rel, kappa)
     del Ug
     rows = np.sort(np.random.default_rng(2).choice(L.m, size=1024, replace=False))

@@ -217,7 +217,7 @@ def test_quantize_edge_cases(m, d, bits, gs, B):
 
 @pytest.mark.parametrize("d", [768, 2048])
 def test_prepare_dead_channels(d):
-    X, _, dead = _edge_inputs(8, d, seed=d)
+    X, _, dead = _edge_inputs(16, d, seed=d)
     H = oracle.hessian(X.numpy())
     Hd = oracle.dampen(H, 0.01)
     Uref = oracle.inverse_upper_cholesky(Hd)

@@ -358,6 +358,41 @@ def test_act_order_equals_obs_recursion_in_that_order(seed, group_size):
     np.testing.assert_allclose(a["scales"], o["scales"], rtol=1e-6)
 
 
+# ------------------------------------------------------------------------------------ inference product
+def test_dequant_matmul_closed_forms():
+    """Codes all at the zero point give Y = 0; codes one level above it give Y = scale * sum(x) per
+    group; a single code at level k gives scale * (k - zero) * x_j (hand-checkable)."""
+    rng = np.random.default_rng(50)
+    m, d, bits, gs = 3, 64, 3, 32
+    scales = np.array([[0.5, 0.25], [1.0, 2.0], [0.125, 4.0]], dtype=np.float32)
+    zeros = np.array([[3, 4], [0, 7], [5, 1]])
+    x = rng.standard_normal((2, d))
+    codes = np.repeat(zeros, gs, axis=1)
+    Y = O.dequant_matmul(O.pack_codes(codes, bits), scales, zeros, bits, gs, d, x)
+    np.testing.assert_array_equal(Y, 0.0)
+    Y = O.dequant_matmul(O.pack_codes(np.minimum(codes + 1, 7), bits), scales, zeros, bits, gs, d, x)
+    for r in range(m):
+        want = sum(float(scales[r, k]) * (min(zeros[r, k] + 1, 7) - zeros[r, k]) * x[:, k * gs:(k + 1) * gs].sum(1)
+                   for k in range(2))
+        np.testing.assert_allclose(Y[:, r], want, rtol=1e-12, atol=1e-12)
+    one = codes.copy()
+    one[1, 40] = 2                               # row 1, group 1 (scale 2, zero 7): level 2 -> 2 * (2 - 7)
+    Y1 = O.dequant_matmul(O.pack_codes(one, bits), scales, zeros, bits, gs, d, x)
+    np.testing.assert_allclose(Y1[:, 1], 2.0 * (2 - 7) * x[:, 40], rtol=1e-12)
+
+
+@pytest.mark.parametrize("group_size", [0, 32])
+def test_dequant_matmul_is_the_layer_product_with_quantized_weights(group_size):
+    rng = np.random.default_rng(51)
+    d, m = 96, 20
+    X = _correlated_x(200, d, rng)
+    W = rng.standard_normal((m, d)) * 0.02
+    res = O.gptq_layer(W, X, bits=4, group_size=group_size, block_size=32)
+    x_in = rng.standard_normal((5, d))
+    Y = O.dequant_matmul(res["packed"], res["scales"], res["zeros"], 4, group_size, d, x_in)
+    np.testing.assert_allclose(Y, x_in @ res["Wq"].T, rtol=1e-12, atol=1e-14)
+
+
 # ------------------------------------------------------------------------------------ mutation check
 def test_planted_mistakes_are_caught():
     """Plant plausible mistakes in what the column loop is given and check a pin fails for each."""
