@@ -107,6 +107,46 @@ class ShardedRunner:
         self.s.run_host(W_h, X_h, out_p, out_s, out_z)
 
 
+def dequant_gemv_figures(g, solver, L, dev, pk, reps: int = 20):
+    """The inference product with this layer's packed weights, one fp16 input row (the step after the
+    path): gptq_dequant_matmul against torch's fp16 matrix-vector product with W, both timed by CUDA
+    events over ``reps`` launches (the packed words and W are larger than L2)."""
+    import torch
+    x = torch.randn(1, L.d, device=dev, dtype=torch.float16)
+    y = torch.empty(1, L.m, device=dev)
+    ws = torch.empty(g.gptq_dequant_matmul_workspace_size(L.m, L.d, 1), dtype=torch.uint8, device=dev)
+    W16 = solver.W.to(torch.float16)
+    xt = x.t().contiguous()
+
+    def ours():
+        g.gptq_dequant_matmul(solver.packed, solver.scales, solver.zeros, L.bits, L.group_size, x, y, ws)
+
+    def fp16():
+        torch.matmul(W16, xt)
+
+    out = {}
+    for name, fn in (("ours", ours), ("fp16", fp16)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        out[name] = e0.elapsed_time(e1) / reps
+    del W16
+    n_groups = 1 if L.group_size == 0 else L.d // L.group_size
+    nbytes = L.m * L.d * L.bits // 8 + 8 * L.m * n_groups + 2 * L.d + 4 * L.m
+    gbs = nbytes / (out["ours"] * 1e-3) / 1e9
+    return {"kernel": "dequant_matmul_kernel + dequant_reduce_kernel", "batch": 1, "x_dtype": "float16",
+            "ms": out["ours"], "algorithmic_bytes": nbytes, "gbs": gbs, "bound": "hbm",
+            "frac": gbs / pk["hbm_gbs"], "peak_source": f"of {pk['source']} HBM copy",
+            "fp16_gemv_ms": out["fp16"], "fp16_gemv": "torch.matmul(W fp16, x) (cuBLAS)",
+            "speedup_vs_fp16": out["fp16"] / out["ours"]}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -456,6 +496,8 @@ def main():
     h2d = W_h.numel() * W_h.element_size() + X_h.numel() * X_h.element_size()
     d2h = sum(t.numel() * t.element_size() for t in (out_p, out_s, out_z))
 
+    gemv = dequant_gemv_figures(g, solver, L, dev, pk) if args.mode == "layers" else None
+
     # denominators: bf16 and HBM measured (MEASURED_PEAKS.json); fp32 FMA measured here by a cuBLAS
     # fp32 GEMM; 3xTF32 derived from the measured bf16 figure and the nominal tf32/bf16 ratio
     fp32_meas = measure_fp32_fma_tflops(dev)
@@ -538,6 +580,8 @@ def main():
                               "(nominal ratio) / 3 MMAs"},
             "end_to_end_roofline_frac_fp32_pipes": roof_fp32_ms / ms_per_step,
             "clocks": clk}
+    if gemv is not None:
+        line["dequant_gemv"] = gemv
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores, blas = cores_info()
         t0 = time.perf_counter()
