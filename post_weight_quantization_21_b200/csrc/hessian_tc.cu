@@ -17,6 +17,9 @@
 //               partial) to global memory.
 // Every mbarrier wait is bounded: on a timeout the kernel records GPTQ_ERR_TIMEOUT, lets the
 // other roles leave, waits (bounded) for its own TMA copies and MMAs in flight, frees TMEM, returns.
+//
+// Orders 512..8192 run the CTA-pair form instead (hessian_pair_kernel, further down): 256 x 256
+// tiles on two SMs with tcgen05.mma.cta_group::2, half the shared-memory traffic per product.
 #include <atomic>
 
 #include "kernels.h"
