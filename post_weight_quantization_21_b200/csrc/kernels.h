@@ -43,17 +43,40 @@ bool tf32x3_map(CUtensorMap* map, const float* base, int64_t rows, int64_t cols,
 gptq_status tf32x3_gemm_launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O, Tf32x3Args a,
                                cudaStream_t stream, int reserve_sms = 0);
 
+// fp32-accurate C -= A B^T on CTA pairs with operands split into tf32 hi / lo beforehand
+// (gemm_tf32x3_pair.cu).  A and B are [rows, 128] K-major panels; C is reduce-added through `out`.
+enum PairKind { kPairSyrk = 0, kPairLazy = 1 };
+struct PairGemmArgs {
+  int kind, tiles;
+  int tiles_n;          // lazy: 256-column tiles
+  int super_n;          // syrk: 256-row super-blocks of the trailing matrix
+  int nk;               // K stages of 32
+  int o_w, o_h;         // output extent (columns, rows)
+  int out_y0, out_x0;   // output origin of tile (0, 0)
+  int skip_diag;        // syrk: leave the first diagonal 128-block to the look-ahead
+  uint32_t idesc;       // set by the launcher
+  int32_t* status;
+};
+bool split_map(CUtensorMap* map, const float* base, int64_t rows);  // [rows, 128] hi or lo panel
+gptq_status split_rows_launch(const float* src, int64_t ld, int64_t rows, float* hi, float* lo, cudaStream_t s);
+gptq_status split_transpose_launch(const float* src, int64_t ld, int64_t cols, float* hi, float* lo,
+                                   cudaStream_t s);
+gptq_status tf32x3_pair_launch(const CUtensorMap& a_hi, const CUtensorMap& a_lo, const CUtensorMap& b_hi,
+                               const CUtensorMap& b_lo, const CUtensorMap& out, PairGemmArgs g, cudaStream_t s,
+                               int reserve_pairs = 0);
+
 // A2 + A3
-size_t prepare_blocked_workspace(int64_t d);
+// with_pair: room for the split panel of the pair-GEMM trailing update (the workspace entry point)
+size_t prepare_blocked_workspace(int64_t d, bool with_pair = true);
 // lookahead: factor the next diagonal block on a library-owned second stream (made once per device)
 gptq_status prepare_blocked_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
-                                   void* workspace, cudaStream_t stream, bool lookahead);
+                                   void* workspace, cudaStream_t stream, bool lookahead, bool pair = true);
 size_t prepare_workspace(int64_t d);
 // the blocked path's tile products run as 3xTF32 tensor-core products; the launch takes exactly this
 // path or fails
 bool prepare_uses_tensor_cores(int64_t d);
 gptq_status prepare_launch(const float* H, int64_t d, float damp, float* U, int32_t* status,
-                           void* workspace, cudaStream_t stream, bool lookahead = true);
+                           void* workspace, cudaStream_t stream, bool lookahead = true, bool pair = true);
 // same, with the scratch in a static device array (d <= GPTQ_PREPARE_STATIC_MAX_D)
 gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* U, int32_t* status,
                                   cudaStream_t stream);

@@ -471,8 +471,8 @@ size_t prepare_workspace(int64_t d) {
 }
 
 gptq_status prepare_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status, void* workspace,
-                           cudaStream_t stream, bool lookahead) {
-  if (d64 > kSmallOrder) return prepare_blocked_launch(H, d64, damp, U, status, workspace, stream, lookahead);
+                           cudaStream_t stream, bool lookahead, bool pair) {
+  if (d64 > kSmallOrder) return prepare_blocked_launch(H, d64, damp, U, status, workspace, stream, lookahead, pair);
   const int d = (int)d64;
   char* ws = static_cast<char*>(workspace);
   PrepArgs a;
@@ -581,9 +581,11 @@ gptq_status prepare_launch_static(const float* H, int64_t d, float damp, float* 
   void* scratch = nullptr;
   gptq_status st = static_scratch(&scratch);
   if (st != GPTQ_OK) return st;
-  if (prepare_workspace(d) > kStaticScratchBytes) return GPTQ_ERR_WORKSPACE;
-  // no look-ahead stream here: this variant creates no CUDA objects, so every launch stays on `stream`
-  return prepare_launch(H, d, damp, U, status, scratch, stream, false);
+  const size_t need = d > kSmallOrder ? prepare_blocked_workspace(d, false) : prepare_workspace(d);
+  if (need > kStaticScratchBytes) return GPTQ_ERR_WORKSPACE;
+  // no look-ahead stream here: this variant creates no CUDA objects, so every launch stays on `stream`;
+  // its scratch holds no split panel, so the trailing updates take the single-CTA tiles
+  return prepare_launch(H, d, damp, U, status, scratch, stream, false, false);
 }
 
 }  // namespace gptq

@@ -457,9 +457,13 @@ __global__ void rotate_kernel(float* __restrict__ P, int d) {
 
 }  // namespace
 
-size_t prepare_blocked_workspace(int64_t d) {
+// header (1 KiB), the inverse diagonal blocks (side), and with_pair: the tf32 hi / lo split of one
+// L panel ([d, 128] each) for the pair-GEMM trailing update
+size_t prepare_blocked_workspace(int64_t d, bool with_pair) {
   const int64_t D = (d + BB - 1) / BB;
-  return kSideOff + (size_t)D * BB * BB * sizeof(float);
+  size_t n = kSideOff + (size_t)D * BB * BB * sizeof(float);
+  if (with_pair) n = align_up(n, 256) + 2 * align_up((size_t)d * BB * sizeof(float), 256);
+  return n;
 }
 
 namespace {
@@ -489,7 +493,7 @@ bool tc_maps(TcMaps& m, const float* P, const float* side, int d, int D) {
 }  // namespace
 
 gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, float* U, int32_t* status, void* workspace,
-                                   cudaStream_t s, bool lookahead) {
+                                   cudaStream_t s, bool lookahead, bool pair) {
   const int d = (int)d64;
   const int D = (d + BB - 1) / BB;
   char* ws = static_cast<char*>(workspace);
@@ -504,6 +508,18 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
   // U is 16-byte aligned (checked by the entry points), the scratch 256-byte aligned and d % 4 == 0 on
   // this path, so the maps encode unless the driver call itself fails
   if (tc && !tc_maps(maps, U, side, d, D)) return GPTQ_ERR_CUDA;
+  // the trailing updates on CTA pairs from the split L panel (workspace entry point, tensor-core path)
+  const bool use_pair = tc && pair;
+  float* Lh = nullptr;
+  float* Ll = nullptr;
+  CUtensorMap mLh, mLl, mP;
+  if (use_pair) {
+    const size_t off = align_up(kSideOff + (size_t)D * BB * BB * sizeof(float), 256);
+    Lh = reinterpret_cast<float*>(ws + off);
+    Ll = reinterpret_cast<float*>(ws + off + align_up((size_t)d * BB * sizeof(float), 256));
+    if (!split_map(&mLh, Lh, d) || !split_map(&mLl, Ll, d) || !tf32x3_map(&mP, U, d, d, d, 32))
+      return GPTQ_ERR_CUDA;
+  }
   std::unique_lock<std::mutex> hold(g_lookahead_mu, std::defer_lock);
   LookAhead* la = nullptr;
   if (lookahead && dev < 64) {
@@ -549,7 +565,37 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
       GPTQ_CUDA_TRY(cudaEventRecord(la->fork, s));
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
     }
-    if (tc) {
+    if (tc && use_pair) {
+      // L(r, p) for the trailing rows, split into tf32 hi / lo once; then the pair-GEMM update of every
+      // block of the trailing lower triangle (the next diagonal block too unless the look-ahead does it)
+      const int64_t rows = d - (int64_t)(p + 1) * BB;
+      if ((st = split_rows_launch(U + (size_t)(p + 1) * BB * d + (size_t)p * BB, d, rows, Lh, Ll, s)) != GPTQ_OK)
+        return st;
+      PairGemmArgs pg{};
+      pg.kind = kPairSyrk;
+      pg.super_n = (below + 1) / 2;
+      pg.tiles = pg.super_n * (pg.super_n + 1) / 2;
+      pg.nk = BB / 32;
+      pg.o_w = d;
+      pg.o_h = d;
+      pg.out_y0 = pg.out_x0 = (p + 1) * BB;
+      pg.status = status;
+      if (la != nullptr) {
+        g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = 1, g.p = p, g.skip = 0;
+        if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, fs)) != GPTQ_OK) return st;
+        factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, 0, side, status);
+        GPTQ_LAUNCH_CHECK();
+        GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
+        pg.skip_diag = 1;
+        if ((st = tf32x3_pair_launch(mLh, mLl, mLh, mLl, mP, pg, s, 1)) != GPTQ_OK) return st;
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+      } else {
+        pg.skip_diag = 0;
+        if ((st = tf32x3_pair_launch(mLh, mLl, mLh, mLl, mP, pg, s)) != GPTQ_OK) return st;
+        factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, 0, side, status);
+        GPTQ_LAUNCH_CHECK();
+      }
+    } else if (tc) {
       if (la != nullptr) {
         g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = 1, g.p = p, g.skip = 0;
         if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, fs)) != GPTQ_OK) return st;

@@ -576,9 +576,16 @@ void launch_convert(const void* W, int64_t m, int d, int bits, int gs, float* ww
 // Per-block launches: the column loop of block [i1, i1 + B) for all rows, then the lazy update of the
 // trailing columns, on the tensor cores (3xTF32) unless `fma` asks for the fp32 FMA tile kernel or the
 // buffers are not 16-byte aligned for TMA.
+// The lazy update of 128-column blocks on CTA pairs (gemm_tf32x3_pair.cu): the block's errors and the
+// U panel are split into tf32 hi / lo in these buffers first ([m, 128] and [d, 128] each).
+struct PairBuffers {
+  float *e_hi, *e_lo, *u_hi, *u_lo;
+};
+
 template <int NS>
 gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, int gs, uint8_t* codes,
-                       float* scales, int32_t* zeros, float* err, bool fma, int32_t* status, cudaStream_t s) {
+                       float* scales, int32_t* zeros, float* err, bool fma, int32_t* status, cudaStream_t s,
+                       const PairBuffers* pb) {
   constexpr int B = 32 * NS;
   // lanes per row of the column loop: 8 while that still leaves about 7 warps per SM, else 4
   const bool lpr8 = m <= 6144;
@@ -598,6 +605,11 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
   if (tc && !(tf32x3_map(&mErr, err, m, B, B, 128) && tf32x3_map(&mU, U, d, d, d, 32, true) &&
               tf32x3_map(&mW, ww, m, d, d, 32)))
     return GPTQ_ERR_CUDA;
+  const bool pair = tc && B == 128 && pb != nullptr;
+  CUtensorMap mEh, mEl, mUh, mUl;
+  if (pair && !(split_map(&mEh, pb->e_hi, m) && split_map(&mEl, pb->e_lo, m) && split_map(&mUh, pb->u_hi, d) &&
+                split_map(&mUl, pb->u_lo, d)))
+    return GPTQ_ERR_CUDA;
   Tf32x3Args g{};
   g.kind = kGemmLazy;
   g.epi = kEpiSub;
@@ -615,7 +627,22 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {
-      if (tc) {
+      if (pair) {
+        gptq_status st = split_rows_launch(err, B, m, pb->e_hi, pb->e_lo, s);
+        if (st == GPTQ_OK) st = split_transpose_launch(U + (size_t)i1 * d + i1 + B, d, rest, pb->u_hi, pb->u_lo, s);
+        if (st != GPTQ_OK) return st;
+        PairGemmArgs pg{};
+        pg.kind = kPairLazy;
+        pg.tiles_n = (rest + 255) / 256;
+        pg.tiles = (int)((m + 255) / 256) * pg.tiles_n;
+        pg.nk = B / 32;
+        pg.o_w = d;
+        pg.o_h = (int)m;
+        pg.out_y0 = 0;
+        pg.out_x0 = i1 + B;
+        pg.status = status;
+        if ((st = tf32x3_pair_launch(mEh, mEl, mUh, mUl, mW, pg, s)) != GPTQ_OK) return st;
+      } else if (tc) {
         g.i1 = i1;
         g.i2 = i1 + B;
         g.tiles_n = (rest + 127) / 128;
@@ -658,8 +685,13 @@ gptq_status launch_rows_b(const void* W, int64_t m, int d, const float* U, const
 
 }  // namespace
 
+// fp32 working copy of W, the block's errors, and (128-column blocks on the per-block path) the tf32
+// hi / lo splits of the errors and of the U panel for the pair-GEMM lazy update
 size_t quantize_workspace(int64_t m, int64_t d, int block_size) {
-  return align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * block_size * sizeof(float), 256);
+  size_t n = align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * block_size * sizeof(float), 256);
+  if (block_size == 128 && !quantize_fused(m, d))
+    n += 2 * align_up((size_t)m * 128 * sizeof(float), 256) + 2 * align_up((size_t)d * 128 * sizeof(float), 256);
+  return n;
 }
 
 // One launch per layer with 8 rows per CTA pays off while rows are few (each CTA streams all of U
@@ -697,10 +729,24 @@ gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d
   }
   GPTQ_LAUNCH_CHECK();
   const bool fma = (cfg.flags & GPTQ_FLAG_FP32_FMA) != 0;
+  PairBuffers pb;
+  {
+    size_t off = align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * 128 * sizeof(float), 256);
+    pb.e_hi = reinterpret_cast<float*>(ws + off);
+    off += align_up((size_t)m * 128 * sizeof(float), 256);
+    pb.e_lo = reinterpret_cast<float*>(ws + off);
+    off += align_up((size_t)m * 128 * sizeof(float), 256);
+    pb.u_hi = reinterpret_cast<float*>(ws + off);
+    off += align_up((size_t)d * 128 * sizeof(float), 256);
+    pb.u_lo = reinterpret_cast<float*>(ws + off);
+  }
   switch (cfg.block_size) {
-    case 32: return run_blocks<1>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s);
-    case 64: return run_blocks<2>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s);
-    case 128: return run_blocks<4>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s);
+    case 32: return run_blocks<1>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s,
+                                  nullptr);
+    case 64: return run_blocks<2>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s,
+                                  nullptr);
+    case 128: return run_blocks<4>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s,
+                                   &pb);
     default: return GPTQ_ERR_ARG;
   }
 }
