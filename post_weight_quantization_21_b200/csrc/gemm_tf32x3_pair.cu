@@ -55,15 +55,18 @@ __device__ __forceinline__ void tile_of(int t, const PairGemmArgs& g, int& a_row
     b_row = tn * PT;
     oy = g.out_y0 + tm * PT;
     ox = g.out_x0 + tn * PT;
-  } else {  // syrk: super-tiles (R, C), R >= C, of the trailing matrix (an upper-triangle index, transposed)
-    int C = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
-    while ((C + 1) * (C + 2) / 2 <= t) ++C;
-    while (C * (C + 1) / 2 > t) --C;
-    const int R = C, Cc = t - C * (C + 1) / 2;  // (i = Cc) <= (j = R)
-    a_row = R * PT;
-    b_row = Cc * PT;
+  } else {  // syrk: super-blocks (R, C), C < super_c, C <= R < super_r, column by column
+    int lo = 0, hi = g.super_c - 1;  // the column C with prefix(C) <= t < prefix(C + 1)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((int64_t)mid * g.super_r - (int64_t)mid * (mid - 1) / 2 <= t) lo = mid; else hi = mid - 1;
+    }
+    const int C = lo;
+    const int R = C + (int)(t - ((int64_t)C * g.super_r - (int64_t)C * (C - 1) / 2));
+    a_row = g.row0 + R * PT;
+    b_row = g.row0 + C * PT;
     oy = g.out_y0 + R * PT;
-    ox = g.out_x0 + Cc * PT;
+    ox = g.out_x0 + C * PT;
   }
 }
 
@@ -216,8 +219,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // syrk: only blocks on or below the diagonal, and not the look-ahead's diagonal block
         bool keep = x < g.o_w && y < g.o_h;
         if (g.kind == kPairSyrk) {
-          const int rb = (y - g.out_y0) / HALF, cb = (x - g.out_x0) / HALF;  // 128-blocks of the trailing matrix
-          keep = keep && cb <= rb && !(g.skip_diag && rb == 0 && cb == 0);
+          const int rb = (y - g.out_y0) / HALF, cb = (x - g.out_x0) / HALF;  // 128-blocks of the region
+          keep = keep && cb <= rb && cb < g.cols_blk && !(g.skip_diag && rb == 0 && cb == 0);
         }
         float v[32];
         tmem_ld32(taddr + 32 * ch, v);
@@ -261,9 +264,10 @@ __device__ __forceinline__ float tf32_rn(float x) {
   return __uint_as_float(r);
 }
 
-// hi[r][k], lo[r][k] of src[r * ld + k], k < 128 (rows of a 128-wide panel)
+// hi[r * dld + k], lo[r * dld + k] of src[r * ld + k], k < 128 (rows of a 128-wide panel)
 __global__ void __launch_bounds__(256) split_rows_kernel(const float* __restrict__ src, int64_t ld, int rows,
-                                                         float* __restrict__ hi, float* __restrict__ lo) {
+                                                         float* __restrict__ hi, float* __restrict__ lo,
+                                                         int64_t dld) {
   const int64_t n = (int64_t)rows * (HALF / 4);
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = e / (HALF / 4);
@@ -272,34 +276,36 @@ __global__ void __launch_bounds__(256) split_rows_kernel(const float* __restrict
     float4 h, l;
     h.x = tf32_rn(x.x), h.y = tf32_rn(x.y), h.z = tf32_rn(x.z), h.w = tf32_rn(x.w);
     l.x = tf32_rn(x.x - h.x), l.y = tf32_rn(x.y - h.y), l.z = tf32_rn(x.z - h.z), l.w = tf32_rn(x.w - h.w);
-    *reinterpret_cast<float4*>(hi + r * HALF + c) = h;
-    *reinterpret_cast<float4*>(lo + r * HALF + c) = l;
+    *reinterpret_cast<float4*>(hi + r * dld + c) = h;
+    *reinterpret_cast<float4*>(lo + r * dld + c) = l;
   }
 }
 
-// hi[n][k], lo[n][k] of src[k * ld + n], k < 128, n < cols (a 128-row panel, transposed to K-major)
+// hi[n][k], lo[n][k] of src[k * ld + n], k < k_rows, n < cols: a panel of k_rows rows transposed to
+// K-major ([cols, k_rows], k_rows a multiple of 32)
 __global__ void __launch_bounds__(256) split_transpose_kernel(const float* __restrict__ src, int64_t ld, int cols,
-                                                              float* __restrict__ hi, float* __restrict__ lo) {
+                                                              int k_rows, float* __restrict__ hi,
+                                                              float* __restrict__ lo) {
   __shared__ float tile[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-  for (int nb = blockIdx.x; nb * 32 < cols; nb += gridDim.x) {
-    for (int kb = 0; kb < HALF; kb += 32) {
-      __syncthreads();
+  const int n_nb = (cols + 31) / 32, n_kb = k_rows / 32;
+  for (int64_t w = blockIdx.x; w < (int64_t)n_nb * n_kb; w += gridDim.x) {
+    const int nb = (int)(w / n_kb), kb = (int)(w % n_kb) * 32;
+    __syncthreads();
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        const int k = kb + ty + j, n = nb * 32 + tx;
-        tile[ty + j][tx] = (n < cols) ? src[(int64_t)k * ld + n] : 0.0f;
-      }
-      __syncthreads();
+    for (int j = 0; j < 32; j += 8) {
+      const int k = kb + ty + j, n = nb * 32 + tx;
+      tile[ty + j][tx] = (n < cols) ? src[(int64_t)k * ld + n] : 0.0f;
+    }
+    __syncthreads();
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        const int n = nb * 32 + ty + j, k = kb + tx;
-        if (n < cols) {
-          const float x = tile[tx][ty + j];
-          const float h = tf32_rn(x);
-          hi[(int64_t)n * HALF + k] = h;
-          lo[(int64_t)n * HALF + k] = tf32_rn(x - h);
-        }
+    for (int j = 0; j < 32; j += 8) {
+      const int n = nb * 32 + ty + j, k = kb + tx;
+      if (n < cols) {
+        const float x = tile[tx][ty + j];
+        const float h = tf32_rn(x);
+        hi[(int64_t)n * k_rows + k] = h;
+        lo[(int64_t)n * k_rows + k] = tf32_rn(x - h);
       }
     }
   }
@@ -333,24 +339,27 @@ int pair_slots(int dev) {
 
 }  // namespace
 
-bool split_map(CUtensorMap* map, const float* base, int64_t rows) {
-  // [rows, 128] fp32 K-major operand: boxes of 32 k x 128 rows, 128-byte swizzle
-  return tf32x3_map(map, base, rows, HALF, HALF, HALF);
+bool split_map(CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld) {
+  // [rows, cols] fp32 K-major operand: boxes of 32 k x 128 rows, 128-byte swizzle
+  return tf32x3_map(map, base, rows, cols, ld, HALF);
 }
 
-gptq_status split_rows_launch(const float* src, int64_t ld, int64_t rows, float* hi, float* lo, cudaStream_t s) {
+gptq_status split_rows_launch(const float* src, int64_t ld, int64_t rows, float* hi, float* lo, int64_t dld,
+                              cudaStream_t s) {
   if (rows <= 0) return GPTQ_OK;
   const int64_t n = rows * (HALF / 4);
   const int blocks = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
-  split_rows_kernel<<<blocks, 256, 0, s>>>(src, ld, (int)rows, hi, lo);
+  split_rows_kernel<<<blocks, 256, 0, s>>>(src, ld, (int)rows, hi, lo, dld);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
 
-gptq_status split_transpose_launch(const float* src, int64_t ld, int64_t cols, float* hi, float* lo, cudaStream_t s) {
+gptq_status split_transpose_launch(const float* src, int64_t ld, int64_t cols, int k_rows, float* hi, float* lo,
+                                   cudaStream_t s) {
   if (cols <= 0) return GPTQ_OK;
-  const int blocks = (int)std::min<int64_t>((cols + 31) / 32, 148 * 8);
-  split_transpose_kernel<<<blocks, 256, 0, s>>>(src, ld, (int)cols, hi, lo);
+  const int64_t work = ((cols + 31) / 32) * (k_rows / 32);
+  const int blocks = (int)std::min<int64_t>(work, 148 * 8);
+  split_transpose_kernel<<<blocks, 256, 0, s>>>(src, ld, (int)cols, k_rows, hi, lo);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

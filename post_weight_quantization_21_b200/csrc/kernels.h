@@ -49,7 +49,9 @@ enum PairKind { kPairSyrk = 0, kPairLazy = 1 };
 struct PairGemmArgs {
   int kind, tiles;
   int tiles_n;          // lazy: 256-column tiles
-  int super_n;          // syrk: 256-row super-blocks of the trailing matrix
+  int super_r, super_c; // syrk: 256-row and 256-column super-blocks of the updated region (R >= C)
+  int cols_blk;         // syrk: 128-block columns of the region (a super-block may reach past them)
+  int row0;             // first row of A and of B in the operand maps for super-block 0
   int nk;               // K stages of 32
   int o_w, o_h;         // output extent (columns, rows)
   int out_y0, out_x0;   // output origin of tile (0, 0)
@@ -57,9 +59,13 @@ struct PairGemmArgs {
   uint32_t idesc;       // set by the launcher
   int32_t* status;
 };
-bool split_map(CUtensorMap* map, const float* base, int64_t rows);  // [rows, 128] hi or lo panel
-gptq_status split_rows_launch(const float* src, int64_t ld, int64_t rows, float* hi, float* lo, cudaStream_t s);
-gptq_status split_transpose_launch(const float* src, int64_t ld, int64_t cols, float* hi, float* lo,
+// [rows, cols] hi or lo operand (row stride ld) for the pair GEMM
+bool split_map(CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld);
+// rows x 128 panel (row stride ld) -> hi / lo (row stride dld)
+gptq_status split_rows_launch(const float* src, int64_t ld, int64_t rows, float* hi, float* lo, int64_t dld,
+                              cudaStream_t s);
+// k_rows x cols panel (row stride ld) -> hi / lo [cols, k_rows] (K-major)
+gptq_status split_transpose_launch(const float* src, int64_t ld, int64_t cols, int k_rows, float* hi, float* lo,
                                    cudaStream_t s);
 gptq_status tf32x3_pair_launch(const CUtensorMap& a_hi, const CUtensorMap& a_lo, const CUtensorMap& b_hi,
                                const CUtensorMap& b_lo, const CUtensorMap& out, PairGemmArgs g, cudaStream_t s,

@@ -457,12 +457,19 @@ __global__ void rotate_kernel(float* __restrict__ P, int d) {
 
 }  // namespace
 
-// header (1 KiB), the inverse diagonal blocks (side), and with_pair: the tf32 hi / lo split of one
-// L panel ([d, 128] each) for the pair-GEMM trailing update
+// Two-level trailing update on the pair path: panels are grouped in outer blocks of kOuterPanels.
+// After panel p, the update reaches only the columns of p's outer block (K = 128); after an outer
+// block's last panel, its L columns (K = 1024) update everything to its right at once.  In exact
+// arithmetic every block P(r, c) still receives every earlier panel's term before it is used; the
+// trailing matrix is read and written once per outer block instead of once per panel.
+constexpr int kOuterPanels = 8;
+
+// header (1 KiB), the inverse diagonal blocks (side), and with_pair: the tf32 hi / lo split of an
+// outer block's L columns ([d, 1024] each) for the pair-GEMM trailing updates
 size_t prepare_blocked_workspace(int64_t d, bool with_pair) {
   const int64_t D = (d + BB - 1) / BB;
   size_t n = kSideOff + (size_t)D * BB * BB * sizeof(float);
-  if (with_pair) n = align_up(n, 256) + 2 * align_up((size_t)d * BB * sizeof(float), 256);
+  if (with_pair) n = align_up(n, 256) + 2 * align_up((size_t)d * kOuterPanels * BB * sizeof(float), 256);
   return n;
 }
 
@@ -510,14 +517,15 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
   if (tc && !tc_maps(maps, U, side, d, D)) return GPTQ_ERR_CUDA;
   // the trailing updates on CTA pairs from the split L panel (workspace entry point, tensor-core path)
   const bool use_pair = tc && pair;
+  constexpr int KO = kOuterPanels * BB;  // row stride of the split L columns
   float* Lh = nullptr;
   float* Ll = nullptr;
   CUtensorMap mLh, mLl, mP;
   if (use_pair) {
     const size_t off = align_up(kSideOff + (size_t)D * BB * BB * sizeof(float), 256);
     Lh = reinterpret_cast<float*>(ws + off);
-    Ll = reinterpret_cast<float*>(ws + off + align_up((size_t)d * BB * sizeof(float), 256));
-    if (!split_map(&mLh, Lh, d) || !split_map(&mLl, Ll, d) || !tf32x3_map(&mP, U, d, d, d, 32))
+    Ll = reinterpret_cast<float*>(ws + off + align_up((size_t)d * KO * sizeof(float), 256));
+    if (!split_map(&mLh, Lh, d, KO, KO) || !split_map(&mLl, Ll, d, KO, KO) || !tf32x3_map(&mP, U, d, d, d, 32))
       return GPTQ_ERR_CUDA;
   }
   std::unique_lock<std::mutex> hold(g_lookahead_mu, std::defer_lock);
@@ -566,32 +574,59 @@ gptq_status prepare_blocked_launch(const float* H, int64_t d64, float damp, floa
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
     }
     if (tc && use_pair) {
-      // L(r, p) for the trailing rows, split into tf32 hi / lo once; then the pair-GEMM update of every
-      // block of the trailing lower triangle (the next diagonal block too unless the look-ahead does it)
+      // L(r, p) of the trailing rows, split into tf32 hi / lo into the outer block's slot p % 8 (rows
+      // keep their absolute index); then the pair-GEMM updates of the two levels
+      const int o0 = p / kOuterPanels * kOuterPanels, pend = std::min(o0 + kOuterPanels, D);
+      const int j = p - o0;
       const int64_t rows = d - (int64_t)(p + 1) * BB;
-      if ((st = split_rows_launch(U + (size_t)(p + 1) * BB * d + (size_t)p * BB, d, rows, Lh, Ll, s)) != GPTQ_OK)
+      const size_t roff = (size_t)(p + 1) * BB * KO + (size_t)j * BB;
+      if ((st = split_rows_launch(U + (size_t)(p + 1) * BB * d + (size_t)p * BB, d, rows, Lh + roff, Ll + roff, KO,
+                                  s)) != GPTQ_OK)
         return st;
+      const bool boundary = p + 1 == pend;  // p closes its outer block
       PairGemmArgs pg{};
       pg.kind = kPairSyrk;
-      pg.super_n = (below + 1) / 2;
-      pg.tiles = pg.super_n * (pg.super_n + 1) / 2;
-      pg.nk = BB / 32;
       pg.o_w = d;
       pg.o_h = d;
-      pg.out_y0 = pg.out_x0 = (p + 1) * BB;
+      pg.out_y0 = pg.out_x0 = pg.row0 = (p + 1) * BB;
       pg.status = status;
-      if (la != nullptr) {
-        g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = 1, g.p = p, g.skip = 0;
-        if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, fs)) != GPTQ_OK) return st;
-        factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, 0, side, status);
-        GPTQ_LAUNCH_CHECK();
-        GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
-        pg.skip_diag = 1;
-        if ((st = tf32x3_pair_launch(mLh, mLl, mLh, mLl, mP, pg, s, 1)) != GPTQ_OK) return st;
-        GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+      if (!boundary) {
+        // inner: rows below p, the columns of p's outer block after p; K = 128 (panel p)
+        CUtensorMap mSh, mSl;
+        if (!split_map(&mSh, Lh + (size_t)j * BB, d, BB, KO) || !split_map(&mSl, Ll + (size_t)j * BB, d, BB, KO))
+          return GPTQ_ERR_CUDA;
+        pg.cols_blk = pend - p - 1;
+        pg.super_r = (below + 1) / 2;
+        pg.super_c = (pg.cols_blk + 1) / 2;
+        pg.tiles = pg.super_c * pg.super_r - pg.super_c * (pg.super_c - 1) / 2;
+        pg.nk = BB / 32;
+        if (la != nullptr) {
+          g.kind = kGemmSyrk, g.epi = kEpiSub, g.b_mn = 0, g.tiles = 1, g.p = p, g.skip = 0;
+          if ((st = tf32x3_gemm_launch(maps.p128, maps.p128, maps.p32, g, fs)) != GPTQ_OK) return st;
+          factor_kernel<<<1, 256, kFactorSmem, fs>>>(U, d, p + 1, 0, side, status);
+          GPTQ_LAUNCH_CHECK();
+          GPTQ_CUDA_TRY(cudaEventRecord(la->join, fs));
+          pg.skip_diag = 1;
+          if ((st = tf32x3_pair_launch(mSh, mSl, mSh, mSl, mP, pg, s, 1)) != GPTQ_OK) return st;
+          GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, la->join, 0));
+        } else {
+          pg.skip_diag = 0;
+          if ((st = tf32x3_pair_launch(mSh, mSl, mSh, mSl, mP, pg, s)) != GPTQ_OK) return st;
+          factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, 0, side, status);
+          GPTQ_LAUNCH_CHECK();
+        }
       } else {
+        // outer: everything right of the outer block, K = the outer block's columns; the next diagonal
+        // block needs all of them, so it is factored after this update (no look-ahead here)
+        const int kcols = (pend - o0) * BB;
+        CUtensorMap mOh, mOl;
+        if (!split_map(&mOh, Lh, d, kcols, KO) || !split_map(&mOl, Ll, d, kcols, KO)) return GPTQ_ERR_CUDA;
+        pg.cols_blk = below;
+        pg.super_r = pg.super_c = (below + 1) / 2;
+        pg.tiles = pg.super_r * (pg.super_r + 1) / 2;
+        pg.nk = kcols / 32;
         pg.skip_diag = 0;
-        if ((st = tf32x3_pair_launch(mLh, mLl, mLh, mLl, mP, pg, s)) != GPTQ_OK) return st;
+        if ((st = tf32x3_pair_launch(mOh, mOl, mOh, mOl, mP, pg, s)) != GPTQ_OK) return st;
         factor_kernel<<<1, 256, kFactorSmem, s>>>(U, d, p + 1, 0, side, status);
         GPTQ_LAUNCH_CHECK();
       }

@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, 
                                                       int group_size, uint8_t* __restrict__ codes,
                                                       float* __restrict__ scales,
                                                       int32_t* __restrict__ zeros,
-                                                      float* __restrict__ err_out) {
+                                                      float* __restrict__ err_out, int err_ld) {
   constexpr int B = LPR * C;
   constexpr int CS = ((C + 4) / 4) % 2 == 1 ? C + 4 : C + 8;  // chunk stride: an odd number of 16-byte granules
   constexpr int RS = LPR * CS;                                  // row stride
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, 
   uint8_t* crow = codes + row * d + i1 + sub * C;
 #pragma unroll
   for (int q = 0; q < C / 4; ++q) reinterpret_cast<uint32_t*>(crow)[q] = cw[q];
-  float* erow = err_out + row * B + sub * C;
+  float* erow = err_out + row * err_ld + sub * C;
 #pragma unroll
   for (int q = 0; q < C / 4; ++q)
     *reinterpret_cast<float4*>(erow + 4 * q) = make_float4(er[4 * q], er[4 * q + 1], er[4 * q + 2], er[4 * q + 3]);
@@ -576,8 +576,15 @@ void launch_convert(const void* W, int64_t m, int d, int bits, int gs, float* ww
 // Per-block launches: the column loop of block [i1, i1 + B) for all rows, then the lazy update of the
 // trailing columns, on the tensor cores (3xTF32) unless `fma` asks for the fp32 FMA tile kernel or the
 // buffers are not 16-byte aligned for TMA.
-// The lazy update of 128-column blocks on CTA pairs (gemm_tf32x3_pair.cu): the block's errors and the
-// U panel are split into tf32 hi / lo in these buffers first ([m, 128] and [d, 128] each).
+// The lazy update of 128-column blocks on CTA pairs (gemm_tf32x3_pair.cu), in two levels.  Columns
+// are grouped in outer blocks of kOuter = 1024 (eight blocks).  After each block's column loop its
+// errors update the remaining columns of the same outer block (K = 128); after the outer block's last
+// block, the outer block's errors (Err [m, 1024]) update all later columns at once (K = 1024).  In
+// exact arithmetic this is the same sum as one update per block (each column still receives every
+// earlier block's term before its own block runs); it reads and writes the trailing W once per outer
+// block instead of once per block.  Errors and U panels are split into tf32 hi / lo first:
+// err/e_hi/e_lo [m, 1024], u_hi/u_lo [d, 1024] (or [n, 128] for the inner updates).
+constexpr int kOuter = 1024;
 struct PairBuffers {
   float *e_hi, *e_lo, *u_hi, *u_lo;
 };
@@ -606,10 +613,29 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
               tf32x3_map(&mW, ww, m, d, d, 32)))
     return GPTQ_ERR_CUDA;
   const bool pair = tc && B == 128 && pb != nullptr;
-  CUtensorMap mEh, mEl, mUh, mUl;
-  if (pair && !(split_map(&mEh, pb->e_hi, m) && split_map(&mEl, pb->e_lo, m) && split_map(&mUh, pb->u_hi, d) &&
-                split_map(&mUl, pb->u_lo, d)))
+  // outer blocks of 1024 columns when every group lies inside one (a group's grid reads its later
+  // columns at the group start, so those must have received every earlier update), else 128
+  const int outer = (pair && (gs == 0 || kOuter % gs == 0)) ? kOuter : B;
+  const int err_ld = pair ? kOuter : B;  // the err buffer holds an outer block's errors on the pair path
+  CUtensorMap mEh, mEl, mUh, mUl, mUin_h, mUin_l;
+  if (pair && !(split_map(&mEh, pb->e_hi, m, kOuter, kOuter) && split_map(&mEl, pb->e_lo, m, kOuter, kOuter) &&
+                split_map(&mUh, pb->u_hi, d, outer, outer) && split_map(&mUl, pb->u_lo, d, outer, outer) &&
+                split_map(&mUin_h, pb->u_hi, d, B, B) && split_map(&mUin_l, pb->u_lo, d, B, B)))
     return GPTQ_ERR_CUDA;
+  auto pair_update = [&](const CUtensorMap& a_hi, const CUtensorMap& a_lo, const CUtensorMap& b_hi,
+                         const CUtensorMap& b_lo, int c0, int c1, int K) -> gptq_status {
+    PairGemmArgs pg{};
+    pg.kind = kPairLazy;
+    pg.tiles_n = (c1 - c0 + 255) / 256;
+    pg.tiles = (int)((m + 255) / 256) * pg.tiles_n;
+    pg.nk = K / 32;
+    pg.o_w = c1;
+    pg.o_h = (int)m;
+    pg.out_y0 = 0;
+    pg.out_x0 = c0;
+    pg.status = status;
+    return tf32x3_pair_launch(a_hi, a_lo, b_hi, b_lo, mW, pg, s);
+  };
   Tf32x3Args g{};
   g.kind = kGemmLazy;
   g.epi = kEpiSub;
@@ -620,28 +646,44 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
   g.status = status;
   const int tiles_m = (int)((m + 127) / 128);
   for (int i1 = 0; i1 < d; i1 += B) {
+    const int o0 = pair ? i1 / outer * outer : i1;           // start of this block's outer block
+    const int slot = i1 - o0;                                 // its column offset in the outer block
+    float* err_b = err + slot;                                // this block's errors (row stride err_ld)
     if (lpr8)
-      colloop_kernel<C8, 8><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
+      colloop_kernel<C8, 8><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err_b,
+                                                        err_ld);
     else
-      colloop_kernel<C4, 4><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err);
+      colloop_kernel<C4, 4><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err_b,
+                                                        err_ld);
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {
       if (pair) {
-        gptq_status st = split_rows_launch(err, B, m, pb->e_hi, pb->e_lo, s);
-        if (st == GPTQ_OK) st = split_transpose_launch(U + (size_t)i1 * d + i1 + B, d, rest, pb->u_hi, pb->u_lo, s);
+        const int oend = std::min(o0 + outer, d);
+        gptq_status st = split_rows_launch(err_b, err_ld, m, pb->e_hi + slot, pb->e_lo + slot, kOuter, s);
         if (st != GPTQ_OK) return st;
-        PairGemmArgs pg{};
-        pg.kind = kPairLazy;
-        pg.tiles_n = (rest + 255) / 256;
-        pg.tiles = (int)((m + 255) / 256) * pg.tiles_n;
-        pg.nk = B / 32;
-        pg.o_w = d;
-        pg.o_h = (int)m;
-        pg.out_y0 = 0;
-        pg.out_x0 = i1 + B;
-        pg.status = status;
-        if ((st = tf32x3_pair_launch(mEh, mEl, mUh, mUl, mW, pg, s)) != GPTQ_OK) return st;
+        if (i1 + B < oend) {  // the rest of this outer block, K = 128 (this block's errors)
+          CUtensorMap mEbh, mEbl;
+          if (!split_map(&mEbh, pb->e_hi + slot, m, B, kOuter) || !split_map(&mEbl, pb->e_lo + slot, m, B, kOuter))
+            return GPTQ_ERR_CUDA;
+          st = split_transpose_launch(U + (size_t)i1 * d + i1 + B, d, oend - (i1 + B), B, pb->u_hi, pb->u_lo, s);
+          if (st == GPTQ_OK) st = pair_update(mEbh, mEbl, mUin_h, mUin_l, i1 + B, oend, B);
+          if (st != GPTQ_OK) return st;
+        }
+        if (i1 + B == oend && oend < d) {  // the outer block is done: every later column, K = outer
+          st = split_transpose_launch(U + (size_t)o0 * d + oend, d, d - oend, outer, pb->u_hi, pb->u_lo, s);
+          if (st == GPTQ_OK) {
+            if (outer == kOuter) {
+              st = pair_update(mEh, mEl, mUh, mUl, oend, d, kOuter);
+            } else {  // one block per outer block: its errors sit at slot 0 with row stride kOuter
+              CUtensorMap mEbh, mEbl;
+              if (!split_map(&mEbh, pb->e_hi, m, B, kOuter) || !split_map(&mEbl, pb->e_lo, m, B, kOuter))
+                return GPTQ_ERR_CUDA;
+              st = pair_update(mEbh, mEbl, mUh, mUl, oend, d, B);
+            }
+          }
+          if (st != GPTQ_OK) return st;
+        }
       } else if (tc) {
         g.i1 = i1;
         g.i2 = i1 + B;
@@ -685,12 +727,15 @@ gptq_status launch_rows_b(const void* W, int64_t m, int d, const float* U, const
 
 }  // namespace
 
-// fp32 working copy of W, the block's errors, and (128-column blocks on the per-block path) the tf32
-// hi / lo splits of the errors and of the U panel for the pair-GEMM lazy update
+// fp32 working copy of W, the block's errors, and (128-column blocks on the per-block path) an outer
+// block's errors with their tf32 hi / lo splits and the split U panels of the two-level lazy update
+bool pair_lazy_layout(int64_t m, int64_t d, int block_size) { return block_size == 128 && !quantize_fused(m, d); }
+
 size_t quantize_workspace(int64_t m, int64_t d, int block_size) {
-  size_t n = align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * block_size * sizeof(float), 256);
-  if (block_size == 128 && !quantize_fused(m, d))
-    n += 2 * align_up((size_t)m * 128 * sizeof(float), 256) + 2 * align_up((size_t)d * 128 * sizeof(float), 256);
+  const int err_w = pair_lazy_layout(m, d, block_size) ? kOuter : block_size;
+  size_t n = align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * err_w * sizeof(float), 256);
+  if (pair_lazy_layout(m, d, block_size))
+    n += 2 * align_up((size_t)m * kOuter * sizeof(float), 256) + 2 * align_up((size_t)d * kOuter * sizeof(float), 256);
   return n;
 }
 
@@ -730,14 +775,15 @@ gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d
   GPTQ_LAUNCH_CHECK();
   const bool fma = (cfg.flags & GPTQ_FLAG_FP32_FMA) != 0;
   PairBuffers pb;
-  {
-    size_t off = align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * 128 * sizeof(float), 256);
+  const bool pair_layout = pair_lazy_layout(m, d, cfg.block_size);
+  if (pair_layout) {
+    size_t off = align_up((size_t)m * d * sizeof(float), 256) + align_up((size_t)m * kOuter * sizeof(float), 256);
     pb.e_hi = reinterpret_cast<float*>(ws + off);
-    off += align_up((size_t)m * 128 * sizeof(float), 256);
+    off += align_up((size_t)m * kOuter * sizeof(float), 256);
     pb.e_lo = reinterpret_cast<float*>(ws + off);
-    off += align_up((size_t)m * 128 * sizeof(float), 256);
+    off += align_up((size_t)m * kOuter * sizeof(float), 256);
     pb.u_hi = reinterpret_cast<float*>(ws + off);
-    off += align_up((size_t)d * 128 * sizeof(float), 256);
+    off += align_up((size_t)d * kOuter * sizeof(float), 256);
     pb.u_lo = reinterpret_cast<float*>(ws + off);
   }
   switch (cfg.block_size) {
@@ -746,7 +792,7 @@ gptq_status quantize_launch(const void* W, int32_t w_dtype, int64_t m, int64_t d
     case 64: return run_blocks<2>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s,
                                   nullptr);
     case 128: return run_blocks<4>(ww, m, d, U, cfg.bits, cfg.group_size, codes, scales, zeros, err, fma, status, s,
-                                   &pb);
+                                   pair_layout ? &pb : nullptr);
     default: return GPTQ_ERR_ARG;
   }
 }

@@ -56,7 +56,10 @@ def test_static_prepare_matches_workspace_prepare(d):
         assert code == g.GPTQ_OK, (code, detail)
         got = U.double().cpu().numpy()
         rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
-        assert rel <= U_REL, rel
+        # above d = 1024 the two entry points group the trailing updates differently (the workspace
+        # entry point updates in two levels on CTA pairs), so they agree to fp32 rounding amplified
+        # by the condition number: the prepare tests' bound
+        assert rel <= (U_REL if d <= 1024 else o_tol), (rel, o_tol)
         assert np.all(np.tril(got, -1) == 0.0)
         rel_o = np.linalg.norm(got - Uo) / np.linalg.norm(Uo)
         assert rel_o <= o_tol, (rel_o, kappa)
