@@ -43,6 +43,9 @@ def parse():
                    help="N > 1: 'layers' = each rank solves its own layer (weak scaling); 'sharded' = one layer "
                         "split across the ranks (tokens for H + all-reduce, rows for the solve; strong scaling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--pipeline", action="store_true",
+                   help="time the sequential block pipeline instead (OPT-125M-like synthetic blocks, 128 x 2048 "
+                        "calibration tokens): one JSON line of its own")
     p.add_argument("--e2e-steps", type=int, default=None,
                    help="end-to-end steps (default: 10, or 3 on layers whose step takes over 0.5 s)")
     return p.parse_args()
@@ -391,12 +394,42 @@ def config_of(L):
             "l2": f"inputs larger than L2: X = {xb / 1e9:.2f} GB streamed from HBM every step"}
 
 
+def run_pipeline(args):
+    """Sequential quantization of synthetic OPT-125M-like blocks (d 768, 12 heads, ffn 3072) on 128 x 2048
+    calibration tokens: per block, the full-precision forward with the Hessians of its four linear
+    inputs, the six layer solves, and the forward with the dequantized weights."""
+    import torch
+    from post_weight_quantization_21_b200 import pipeline as P
+    cfg = P.BlockConfig(d_model=768, n_heads=12, d_ffn=3072, seq_len=2048, bits=4, group_size=0, block_size=128)
+    dev = torch.device("cuda", 0)
+    X = torch.randn(128 * cfg.seq_len, cfg.d_model, device=dev, generator=torch.Generator(device=dev).manual_seed(0))
+    X = X.to(torch.bfloat16)
+    bq = P.BlockQuantizer(cfg, device=dev, chunk_seqs=16)
+    x = X
+    for b in range(args.warmup):
+        _, x = bq.quantize_block(P.make_block(cfg, seed=b, device=dev), x)
+    times = []
+    for b in range(args.steps):
+        _, x = bq.quantize_block(P.make_block(cfg, seed=1000 + b, device=dev), x)
+        times.append(dict(bq.timing))
+    ms = {k: statistics.mean(t[k] for t in times) for k in times[0]}
+    total = sum(ms.values())
+    weights = sum(cfg.shape(n)[0] * cfg.shape(n)[1] for n in P.LINEARS)
+    print(json.dumps({"metric": "sequential block pipeline: ms per block", "value": total, "unit": "ms",
+                      "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+                      "split_ms": ms, "weights_per_s": weights / (total * 1e-3),
+                      "config": {"workload": "synthetic OPT-125M-like decoder block", "d_model": 768, "n_heads": 12,
+                                 "d_ffn": 3072, "tokens": 128 * 2048, "bits": 4, "group_size": 0}}), flush=True)
+
+
 def main():
     args = parse()
     from post_weight_quantization_21_b200 import workloads as wl
     L = wl.LAYERS[args.layer]
     if args.impl == "reference":
         return run_reference(args, L)
+    if args.pipeline:
+        return run_pipeline(args)
 
     import torch
     import torch.distributed as dist

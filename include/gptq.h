@@ -256,6 +256,19 @@ GPTQ_API gptq_status gptq_dequant_matmul(const int32_t* packed, const float* sca
 GPTQ_API size_t gptq_dequant_matmul_workspace_size(int64_t m, int64_t d, int64_t batch);
 
 /* ------------------------------------------------------------------------------------------
+ * The dequantized weights What[r, j] = scale[r, g(j)] * (q[r, j] - zero[r, g(j)]) as a dense matrix
+ * (the values a quantized layer computes with; FDE breakdown section 01 and figure step 1: the
+ * weights on the b-bit grid), e.g. for running a quantized block forward to produce the next
+ * block's calibration inputs.
+ *   packed [m, d*bits/32] int32 (gptq_pack), scales / zeros [m, n_groups]; W_hat [m, d] row-major
+ *   in out_dtype (BF16 / FP16 rounded to nearest from the fp32 product, or FP32).
+ *   Requires d % 32 == 0, bits in {2, 3, 4}, group_size 0 or a multiple of 32 dividing d.
+ * ------------------------------------------------------------------------------------------ */
+GPTQ_API gptq_status gptq_dequantize(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m,
+                                     int64_t d, int32_t bits, int32_t group_size, void* W_hat, int32_t out_dtype,
+                                     void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * Status helpers.
  * gptq_read_status: synchronizes `stream`, copies the device status word to the host, returns the
  * code it holds (GPTQ_OK if clear) and stores its detail (e.g. the failing pivot) in *detail when

@@ -25,7 +25,7 @@ __all__ = [
     "gptq_prepare_workspace_size", "gptq_prepare_uinv_static", "gptq_quantize_layer", "gptq_quantize_workspace_size", "gptq_pack",
     "gptq_read_status", "gptq_status_string", "gptq_kernel_launches", "gptq_tensor_core_phases", "LayerSolver", "LIB_PATH", "ABI_FUNCTIONS",
     "gptq_act_order", "gptq_quantize_layer_act_order", "gptq_quantize_act_order_workspace_size", "act_order_group_index",
-    "gptq_dequant_matmul", "gptq_dequant_matmul_workspace_size",
+    "gptq_dequant_matmul", "gptq_dequant_matmul_workspace_size", "gptq_dequantize",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -63,6 +63,7 @@ ABI_FUNCTIONS = {
     "gptq_test_hessian_timeout": (None, [_i64]),
     "gptq_dequant_matmul": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _i32, _i64, _vp, _vp, _sz, _vp]),
     "gptq_dequant_matmul_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "gptq_dequantize": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _i32, _vp]),
     "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
     "gptq_status_string": (ctypes.c_char_p, [_i32]),
     "gptq_abi_version": (_i32, []),
@@ -250,6 +251,16 @@ def gptq_dequant_matmul(packed: torch.Tensor, scales: torch.Tensor, zeros: torch
                                    _DTYPES[X.dtype], batch, _ptr(Y), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "gptq_dequant_matmul")
+
+
+def gptq_dequantize(packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int, group_size: int,
+                    W_hat: torch.Tensor, stream=None):
+    """W_hat [m, d] (fp16 / bf16 / fp32) = the dequantized weights of the packed codes."""
+    for t, n in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (W_hat, "W_hat")):
+        _contig(t, n)
+    m, d = W_hat.shape
+    _check(lib().gptq_dequantize(_ptr(packed), _ptr(scales), _ptr(zeros), m, d, bits, group_size, _ptr(W_hat),
+                                 _DTYPES[W_hat.dtype], _stream(stream)), "gptq_dequantize")
 
 
 def gptq_tensor_core_phases(m: int, d: int, n_tokens: int, x_dtype, bits: int, group_size: int = 0,

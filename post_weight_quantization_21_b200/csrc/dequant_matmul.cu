@@ -51,6 +51,15 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
   }
 }
 
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
 // 1 + q_j / 2^BITS for code j (0..31) of a unit held in w[0..BITS-1].
 template <int BITS>
 __device__ __forceinline__ float decode(const uint32_t (&w)[BITS], const int j) {
@@ -206,11 +215,62 @@ gptq_status launch_typed(const int32_t* packed, const float* scales, const int32
   return GPTQ_OK;
 }
 
+// What[r][j] = scale[r][g(j)] * (q[r][j] - zero[r][g(j)]) from the packed words, 32 codes per thread
+template <typename TO, int BITS>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restrict__ packed,
+                                                         const float* __restrict__ scales,
+                                                         const int32_t* __restrict__ zeros, int64_t m, int d,
+                                                         int group_size, TO* __restrict__ out) {
+  const int units = d >> 5, ng = group_size ? d / group_size : 1, upg = group_size ? group_size >> 5 : units;
+  const int wpr = units * BITS;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < m * units; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / units;
+    const int u = (int)(e % units);
+    uint32_t w[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) w[k] = packed[r * wpr + (int64_t)u * BITS + k];
+    const float sc = scales[r * ng + u / upg], z = (float)zeros[r * ng + u / upg];
+    TO* dst = out + r * d + (int64_t)u * 32;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float q = (decode<BITS>(w, j) - 1.0f) * (float)(1 << BITS);  // exact: q = 2^b (f - 1)
+      dst[j] = from_f32<TO>(sc * (q - z));
+    }
+  }
+}
+
 }  // namespace
 
 size_t dequant_matmul_workspace(int64_t m, int64_t d, int64_t batch) {
   const int64_t tiles = (d / 32 + kUnitsPerTile - 1) / kUnitsPerTile;
   return align_up((size_t)tiles * (size_t)std::min<int64_t>(batch, 4) * m * sizeof(float), 256);
+}
+
+template <typename TO>
+gptq_status dequantize_typed(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m, int64_t d,
+                             int32_t bits, int32_t group_size, void* out, cudaStream_t s) {
+  const uint32_t* pw = reinterpret_cast<const uint32_t*>(packed);
+  const int64_t n = m * (d / 32);
+  const int blocks = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
+  TO* o = static_cast<TO*>(out);
+  switch (bits) {
+    case 2: dequantize_kernel<TO, 2><<<blocks, 256, 0, s>>>(pw, scales, zeros, m, (int)d, group_size, o); break;
+    case 3: dequantize_kernel<TO, 3><<<blocks, 256, 0, s>>>(pw, scales, zeros, m, (int)d, group_size, o); break;
+    case 4: dequantize_kernel<TO, 4><<<blocks, 256, 0, s>>>(pw, scales, zeros, m, (int)d, group_size, o); break;
+    default: return GPTQ_ERR_ARG;
+  }
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+gptq_status dequantize_launch(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m, int64_t d,
+                              int32_t bits, int32_t group_size, void* out, int32_t out_dtype, cudaStream_t s) {
+  switch (out_dtype) {
+    case GPTQ_FP16: return dequantize_typed<__half>(packed, scales, zeros, m, d, bits, group_size, out, s);
+    case GPTQ_BF16: return dequantize_typed<__nv_bfloat16>(packed, scales, zeros, m, d, bits, group_size, out, s);
+    case GPTQ_FP32: return dequantize_typed<float>(packed, scales, zeros, m, d, bits, group_size, out, s);
+    default: return GPTQ_ERR_ARG;
+  }
 }
 
 gptq_status dequant_matmul_launch(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m,

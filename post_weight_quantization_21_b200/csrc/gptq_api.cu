@@ -204,6 +204,18 @@ gptq_status gptq_dequant_matmul(const int32_t* packed, const float* scales, cons
                                      static_cast<cudaStream_t>(stream));
 }
 
+gptq_status gptq_dequantize(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m, int64_t d,
+                            int32_t bits, int32_t group_size, void* W_hat, int32_t out_dtype, void* stream) {
+  if (m <= 0 || d <= 0 || d % 32 || d > kMaxDim || m > kMaxDim * 64 || bits < 2 || bits > 4) return GPTQ_ERR_ARG;
+  if (!valid_dtype(out_dtype)) return GPTQ_ERR_ARG;
+  if (group_size < 0 || (group_size && (group_size % 32 || d % group_size))) return GPTQ_ERR_ARG;
+  if (!packed || !scales || !zeros || !W_hat) return GPTQ_ERR_ARG;
+  if (!aligned(packed, 4) || !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(W_hat, dtype_size(out_dtype)))
+    return GPTQ_ERR_ARG;
+  return gptq::dequantize_launch(packed, scales, zeros, m, d, bits, group_size, W_hat, out_dtype,
+                                 static_cast<cudaStream_t>(stream));
+}
+
 gptq_status gptq_read_status(const int32_t* dev_status, void* stream, int64_t* detail) {
   if (dev_status == nullptr) return GPTQ_ERR_ARG;
   int32_t h[2] = {0, 0};

@@ -113,6 +113,9 @@ gptq_status dequant_matmul_launch(const int32_t* packed, const float* scales, co
                                   int64_t d, int32_t bits, int32_t group_size, const void* X, int32_t x_dtype,
                                   int64_t batch, float* Y, void* workspace, cudaStream_t stream);
 
+gptq_status dequantize_launch(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m, int64_t d,
+                              int32_t bits, int32_t group_size, void* out, int32_t out_dtype, cudaStream_t stream);
+
 // A7
 gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, int32_t* packed,
                         cudaStream_t stream);
