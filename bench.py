@@ -118,11 +118,12 @@ def dequant_gemv_figures(g, solver, L, dev, pk, reps: int = 20):
     x = torch.randn(1, L.d, device=dev, dtype=torch.float16)
     y = torch.empty(1, L.m, device=dev)
     ws = torch.empty(g.gptq_dequant_matmul_workspace_size(L.m, L.d, 1), dtype=torch.uint8, device=dev)
+    st = torch.zeros(2, dtype=torch.int32, device=dev)
     W16 = solver.W.to(torch.float16)
     xt = x.t().contiguous()
 
     def ours():
-        g.gptq_dequant_matmul(solver.packed, solver.scales, solver.zeros, L.bits, L.group_size, x, y, ws)
+        g.gptq_dequant_matmul(solver.packed, solver.scales, solver.zeros, L.bits, L.group_size, x, y, st, ws)
 
     def fp16():
         torch.matmul(W16, xt)

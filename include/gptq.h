@@ -241,18 +241,23 @@ GPTQ_API gptq_status gptq_pack(const uint8_t* codes, int64_t m, int64_t d, int32
  *   packed     [m, d*bits/32] int32 from gptq_pack; scales / zeros [m, n_groups] from
  *              gptq_quantize_layer.  Under act-order the groups follow the quantization order: pass
  *              the codes in that order (codes[:, perm] packed) and X with its columns permuted alike.
- *   X          [batch, d] row-major, BF16 / FP16 / FP32, 16-byte aligned.  1 <= batch <= 1024
- *              (processed four rows at a time).
+ *   X          [batch, d] row-major, BF16 / FP16 / FP32, 16-byte aligned, |x| < 2^100 (inputs are
+ *              pre-scaled by powers of two up to 2^23 inside the kernel).  1 <= batch <= 1024
+ *              (processed four rows at a time).  Every product q x is formed exactly and rounded
+ *              once; the sums are fp32.
  *   Y          [batch, m] fp32 output.
+ *   dev_status int32[2]: cleared at the start of the call; GPTQ_ERR_TIMEOUT if a bounded wait for the
+ *              staged copies of the packed words gave up (d % 128 == 0 stages them in shared memory).
  *   workspace  >= gptq_dequant_matmul_workspace_size(m, d, batch) bytes, 256-byte aligned (partial
  *              sums of the column tiles; the final sum runs in tile order, so results are
  *              deterministic).
- *   Requires d % 32 == 0, bits in {2, 3, 4}, group_size 0 or a multiple of 32 dividing d.
+ *   Requires d % 32 == 0, bits in {2, 3, 4}, group_size 0 or a multiple of 32 dividing d, `packed`
+ *   16-byte aligned.
  * ------------------------------------------------------------------------------------------ */
 GPTQ_API gptq_status gptq_dequant_matmul(const int32_t* packed, const float* scales, const int32_t* zeros,
                                          int64_t m, int64_t d, int32_t bits, int32_t group_size, const void* X,
-                                         int32_t x_dtype, int64_t batch, float* Y, void* workspace,
-                                         size_t workspace_bytes, void* stream);
+                                         int32_t x_dtype, int64_t batch, float* Y, int32_t* dev_status,
+                                         void* workspace, size_t workspace_bytes, void* stream);
 GPTQ_API size_t gptq_dequant_matmul_workspace_size(int64_t m, int64_t d, int64_t batch);
 
 /* ------------------------------------------------------------------------------------------

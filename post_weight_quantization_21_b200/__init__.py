@@ -61,7 +61,8 @@ ABI_FUNCTIONS = {
                                              _vp, _vp, _vp, _sz, _vp]),
     "gptq_quantize_act_order_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(QuantCfg)]),
     "gptq_test_hessian_timeout": (None, [_i64]),
-    "gptq_dequant_matmul": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _i32, _i64, _vp, _vp, _sz, _vp]),
+    "gptq_dequant_matmul": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _i32, _i64, _vp, _vp, _vp, _sz,
+                                   _vp]),
     "gptq_dequant_matmul_workspace_size": (_sz, [_i64, _i64, _i64]),
     "gptq_dequantize": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _i32, _vp]),
     "gptq_read_status": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
@@ -241,14 +242,14 @@ def gptq_dequant_matmul_workspace_size(m: int, d: int, batch: int) -> int:
 
 
 def gptq_dequant_matmul(packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int, group_size: int,
-                        X: torch.Tensor, Y: torch.Tensor, workspace: torch.Tensor, stream=None):
+                        X: torch.Tensor, Y: torch.Tensor, status: torch.Tensor, workspace: torch.Tensor, stream=None):
     """Y [batch, m] (fp32) = X [batch, d] @ What^T, What dequantized on the fly from the packed codes."""
-    for t, n in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (X, "X"), (Y, "Y")):
+    for t, n in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (X, "X"), (Y, "Y"), (status, "status")):
         _contig(t, n)
     m = packed.shape[0]
     batch, d = X.shape
     st = lib().gptq_dequant_matmul(_ptr(packed), _ptr(scales), _ptr(zeros), m, d, bits, group_size, _ptr(X),
-                                   _DTYPES[X.dtype], batch, _ptr(Y), _ptr(workspace),
+                                   _DTYPES[X.dtype], batch, _ptr(Y), _ptr(status), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "gptq_dequant_matmul")
 

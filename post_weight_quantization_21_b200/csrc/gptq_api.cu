@@ -190,18 +190,21 @@ size_t gptq_dequant_matmul_workspace_size(int64_t m, int64_t d, int64_t batch) {
 
 gptq_status gptq_dequant_matmul(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m,
                                 int64_t d, int32_t bits, int32_t group_size, const void* X, int32_t x_dtype,
-                                int64_t batch, float* Y, void* workspace, size_t workspace_bytes, void* stream) {
+                                int64_t batch, float* Y, int32_t* dev_status, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   if (m <= 0 || d <= 0 || d % 32 || d > kMaxDim || m > (int64_t)0x7fffffff - 64 || bits < 2 || bits > 4)
     return GPTQ_ERR_ARG;
   if (batch <= 0 || batch > 1024 || !valid_dtype(x_dtype)) return GPTQ_ERR_ARG;
   if (group_size < 0 || (group_size && (group_size % 32 || d % group_size))) return GPTQ_ERR_ARG;
-  if (!packed || !scales || !zeros || !X || !Y) return GPTQ_ERR_ARG;
-  if (!aligned(packed, 4) || !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(X, 16) || !aligned(Y, 4))
+  if (!packed || !scales || !zeros || !X || !Y || !dev_status) return GPTQ_ERR_ARG;
+  // packed rows start on 16-byte boundaries when d % 128 == 0 (the bulk-copied form needs it)
+  if (!aligned(packed, 16) || !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(X, 16) || !aligned(Y, 4) ||
+      !aligned(dev_status, 4))
     return GPTQ_ERR_ARG;
   const size_t need = gptq::dequant_matmul_workspace(m, d, batch);
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return GPTQ_ERR_WORKSPACE;
-  return gptq::dequant_matmul_launch(packed, scales, zeros, m, d, bits, group_size, X, x_dtype, batch, Y, workspace,
-                                     static_cast<cudaStream_t>(stream));
+  return gptq::dequant_matmul_launch(packed, scales, zeros, m, d, bits, group_size, X, x_dtype, batch, Y, dev_status,
+                                     workspace, static_cast<cudaStream_t>(stream));
 }
 
 gptq_status gptq_dequantize(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m, int64_t d,

@@ -111,7 +111,7 @@ gptq_status quantize_act_order_launch(const void* W, int32_t w_dtype, int64_t m,
 size_t dequant_matmul_workspace(int64_t m, int64_t d, int64_t batch);
 gptq_status dequant_matmul_launch(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m,
                                   int64_t d, int32_t bits, int32_t group_size, const void* X, int32_t x_dtype,
-                                  int64_t batch, float* Y, void* workspace, cudaStream_t stream);
+                                  int64_t batch, float* Y, int32_t* status, void* workspace, cudaStream_t stream);
 
 gptq_status dequantize_launch(const int32_t* packed, const float* scales, const int32_t* zeros, int64_t m, int64_t d,
                               int32_t bits, int32_t group_size, void* out, int32_t out_dtype, cudaStream_t stream);
