@@ -178,8 +178,6 @@ gptq_status gptq_pack(const uint8_t* codes, int64_t m, int64_t d, int32_t bits, 
   if (m <= 0 || d <= 0 || d % 32 || bits < 2 || bits > 4 || !codes || !packed) return GPTQ_ERR_ARG;
   if (!aligned(packed, 4)) return GPTQ_ERR_ARG;
   if (m > kMaxDim * 64 || d > kMaxDim) return GPTQ_ERR_ARG;
-  // one thread per output word: the launch grid must stay within 2^31 - 1 blocks of 256
-  if (m * (d * bits / 32) > (int64_t)0x7fffffff * 256) return GPTQ_ERR_UNSUPPORTED;
   return gptq::pack_launch(codes, m, d, bits, packed, static_cast<cudaStream_t>(stream));
 }
 

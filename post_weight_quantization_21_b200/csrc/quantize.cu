@@ -545,25 +545,46 @@ __global__ void __launch_bounds__(256) lazy_gemm_kernel(float* __restrict__ w, i
   }
 }
 
-// One thread per int32 word of the packed row stream.
-__global__ void pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int d, int bits,
-                            int32_t* __restrict__ packed) {
-  const int wpr = d * bits / 32;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= m * wpr) return;
-  const int64_t row = idx / wpr;
-  const int k = (int)(idx % wpr);
-  const uint32_t mask = (1u << bits) - 1u;
-  const int bit0 = 32 * k;
-  const int j0 = bit0 / bits, j1 = (bit0 + 31) / bits;
-  const uint8_t* cr = codes + row * d;
-  uint32_t word = 0;
-  for (int j = j0; j <= j1 && j < d; ++j) {
-    const uint32_t c = (uint32_t)cr[j] & mask;
-    const int sh = j * bits - bit0;
-    word |= (sh >= 0) ? (c << sh) : (c >> (-sh));
+// One thread per 32-code unit: the unit's 32 code bytes come in as two 16-byte loads (eight 4-byte
+// loads when the codes are only 4-byte aligned, single bytes otherwise) and leave as exactly BITS
+// words, so a warp reads 1 KB and writes 128 * BITS bytes, both contiguous.  HBM-bound: m d (1 + b/8)
+// bytes.  `align`: 16, 4 or 1, the alignment every unit's first code byte has.
+template <int BITS>
+__global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int d, int align,
+                                                   int32_t* __restrict__ packed) {
+  const int upr = d / 32, wpr = upr * BITS;
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < m * upr; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = e / upr;
+    const int u = (int)(e % upr);
+    const uint8_t* src = codes + row * d + (int64_t)u * 32;
+    uint32_t c[8];
+    if (align == 16) {
+      const uint4 lo = __ldg(reinterpret_cast<const uint4*>(src)), hi = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+      c[0] = lo.x, c[1] = lo.y, c[2] = lo.z, c[3] = lo.w, c[4] = hi.x, c[5] = hi.y, c[6] = hi.z, c[7] = hi.w;
+    } else if (align == 4) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) c[k] = __ldg(reinterpret_cast<const uint32_t*>(src) + k);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        c[k] = (uint32_t)src[4 * k] | ((uint32_t)src[4 * k + 1] << 8) | ((uint32_t)src[4 * k + 2] << 16) |
+               ((uint32_t)src[4 * k + 3] << 24);
+    }
+    uint32_t w[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) w[k] = 0u;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t q = (c[j / 4] >> (8 * (j % 4))) & mask;
+      const int bit = BITS * j, k = bit / 32, sh = bit % 32;
+      w[k] |= q << sh;
+      if (sh + BITS > 32) w[k + 1] |= q >> (32 - sh);
+    }
+    int32_t* dst = packed + row * wpr + (int64_t)u * BITS;
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) dst[k] = (int32_t)w[k];
   }
-  packed[idx] = (int32_t)word;
 }
 
 template <typename T>
@@ -801,8 +822,17 @@ gptq_status pack_launch(const uint8_t* codes, int64_t m, int64_t d, int32_t bits
                         cudaStream_t s) {
   const int64_t n = m * (d * bits / 32);
   if (n == 0) return GPTQ_OK;
-  const int threads = 256;
-  pack_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(codes, m, (int)d, bits, packed);
+  const int64_t units = m * (d / 32);
+  const int blocks = (int)std::min<int64_t>((units + 255) / 256, 148 * 16);
+  // d % 32 == 0, so every unit starts as aligned as the codes' base
+  const uintptr_t base = reinterpret_cast<uintptr_t>(codes);
+  const int align = base % 16 == 0 ? 16 : (base % 4 == 0 ? 4 : 1);
+  switch (bits) {
+    case 2: pack_kernel<2><<<blocks, 256, 0, s>>>(codes, m, (int)d, align, packed); break;
+    case 3: pack_kernel<3><<<blocks, 256, 0, s>>>(codes, m, (int)d, align, packed); break;
+    case 4: pack_kernel<4><<<blocks, 256, 0, s>>>(codes, m, (int)d, align, packed); break;
+    default: return GPTQ_ERR_ARG;
+  }
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

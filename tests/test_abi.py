@@ -98,8 +98,8 @@ def test_validation_rejects_bad_arguments_without_a_device(lib):
     assert st == g.GPTQ_ERR_WORKSPACE
     assert lib.gptq_pack(fake, 4, 48, 3, fake, None) == g.GPTQ_ERR_ARG        # d % 32
     assert lib.gptq_pack(fake, 4, 64, 5, fake, None) == g.GPTQ_ERR_ARG        # bits
-    # a grid of one thread per output word past 2^31 - 1 blocks is refused, not launched
-    assert lib.gptq_pack(fake, 1 << 26, 1 << 20, 4, fake, None) == g.GPTQ_ERR_UNSUPPORTED
+    # orders past the documented maximum are refused, not launched
+    assert lib.gptq_pack(fake, 4, (1 << 20) + 32, 4, fake, None) == g.GPTQ_ERR_ARG
     assert lib.gptq_hessian_accumulate(fake, 0, 16, 12, fake, 2.0, 0, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG
     assert lib.gptq_hessian_accumulate(fake, 7, 16, 16, fake, 2.0, 0, fake, fake, 1 << 20, None) == g.GPTQ_ERR_ARG
     other = ctypes.c_void_p(4096)

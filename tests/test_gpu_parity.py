@@ -252,6 +252,19 @@ def test_pack_bit_exact(bits, m, d):
     np.testing.assert_array_equal(got, oracle.pack_codes(codes.numpy().astype(np.int64), bits))
 
 
+@pytest.mark.parametrize("offset", [1, 4, 8])
+def test_pack_codes_at_any_alignment(offset):
+    """The kernel reads a unit's 32 code bytes as 16-, 4- or 1-byte loads by the codes' alignment; the
+    words are the same whichever it takes (codes that carry bits above b are masked)."""
+    m, d, bits = 5, 160, 3
+    codes = torch.randint(0, 256, (m, d), generator=torch.Generator().manual_seed(offset), dtype=torch.uint8)
+    buf = torch.zeros(m * d + 64, dtype=torch.uint8, device=S.dev())
+    view = buf[offset:offset + m * d].view(m, d)
+    view.copy_(codes.to(S.dev()))
+    got = S.pack(view, bits)
+    np.testing.assert_array_equal(got, oracle.pack_codes(codes.numpy().astype(np.int64) & 7, bits))
+
+
 # ------------------------------------------------------------------------------------------ end to end
 def _layer_end_to_end(L, check_h=True):
     W = wl.make_w(L)
