@@ -48,7 +48,53 @@ def parse():
                         "calibration tokens): one JSON line of its own")
     p.add_argument("--e2e-steps", type=int, default=None,
                    help="end-to-end steps (default: 10, or 3 on layers whose step takes over 0.5 s)")
+    p.add_argument("--probe", choices=["hessian", "gemv"], default=None,
+                   help="profiling target, no JSON line: run only the layer's Hessian (gptq_hessian_accumulate) or "
+                        "its dequantizing product (gptq_dequant_matmul, one fp16 row, uniform random codes) "
+                        "--steps times and print the CUDA-event time of each call")
+    p.add_argument("--tokens", type=int, default=None, help="calibration tokens (default: the layer's own)")
     return p.parse_args()
+
+
+def run_probe(args, L):
+    """One kernel of the layer, alone: the command ncu captures are taken on (a few GB on the device)."""
+    import torch
+    import post_weight_quantization_21_b200 as g
+    from post_weight_quantization_21_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    st = torch.zeros(2, dtype=torch.int32, device=dev)
+    if args.probe == "hessian":
+        X = wl.make_x(L, device=dev)
+        H = torch.empty(L.d, L.d, device=dev)
+        ws = torch.empty(max(g.gptq_hessian_workspace_size(L.n_tokens, L.d, X.dtype), 256), dtype=torch.uint8,
+                         device=dev)
+
+        def call():
+            g.gptq_hessian_accumulate(X, H, st, ws, 2.0, False)
+    else:
+        gen = torch.Generator(device="cpu").manual_seed(0)
+        ng = 1 if L.group_size == 0 else L.d // L.group_size
+        packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (L.m, L.d * L.bits // 32), generator=gen,
+                               dtype=torch.int32).to(dev)
+        scales = (torch.rand(L.m, ng, generator=gen) * 0.01).to(dev)
+        zeros = torch.randint(0, 2 ** L.bits, (L.m, ng), generator=gen, dtype=torch.int32).to(dev)
+        x = torch.randn(1, L.d, generator=gen).to(torch.float16).to(dev)
+        y = torch.empty(1, L.m, device=dev)
+        ws = torch.empty(g.gptq_dequant_matmul_workspace_size(L.m, L.d, 1), dtype=torch.uint8, device=dev)
+
+        def call():
+            g.gptq_dequant_matmul(packed, scales, zeros, L.bits, L.group_size, x, y, st, ws)
+    for i in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        code, detail = g.gptq_read_status(st)
+        print(f"{args.probe} {L.name} tokens={L.n_tokens}: {e0.elapsed_time(e1):.3f} ms, status {code}")
+        if code != g.GPTQ_OK:
+            raise g.GPTQError(code, args.probe, detail)
 
 
 def dist_env():
@@ -144,7 +190,7 @@ def dequant_gemv_figures(g, solver, L, dev, pk, reps: int = 20):
     n_groups = 1 if L.group_size == 0 else L.d // L.group_size
     nbytes = L.m * L.d * L.bits // 8 + 8 * L.m * n_groups + 2 * L.d + 4 * L.m
     gbs = nbytes / (out["ours"] * 1e-3) / 1e9
-    return {"kernel": "dequant_matmul_kernel + dequant_reduce_kernel", "batch": 1, "x_dtype": "float16",
+    return {"kernel": "dequant_matmul_staged_kernel + dequant_reduce_kernel", "batch": 1, "x_dtype": "float16",
             "ms": out["ours"], "algorithmic_bytes": nbytes, "gbs": gbs, "bound": "hbm",
             "frac": gbs / pk["hbm_gbs"], "peak_source": f"of {pk['source']} HBM copy",
             "fp16_gemv_ms": out["fp16"], "fp16_gemv": "torch.matmul(W fp16, x) (cuBLAS)",
@@ -427,6 +473,10 @@ def main():
     args = parse()
     from post_weight_quantization_21_b200 import workloads as wl
     L = wl.LAYERS[args.layer]
+    if args.tokens is not None:
+        L = L.with_tokens(args.tokens)
+    if args.probe:
+        return run_probe(args, L)
     if args.impl == "reference":
         return run_reference(args, L)
     if args.pipeline:
