@@ -26,15 +26,13 @@
 namespace gptq {
 namespace {
 
+// Building with GPTQ_DQ_STAGED=0 keeps the register form for every order (for comparisons).
 #ifndef GPTQ_DQ_STAGED
 #define GPTQ_DQ_STAGED 1
 #endif
 constexpr int kWarps = 8;
 // rows per warp: fewer rows for more input rows, so that a thread's sums stay in registers
-#ifndef GPTQ_DQ_RW1
-#define GPTQ_DQ_RW1 8
-#endif
-__host__ __device__ constexpr int rows_per_warp(int nb) { return nb == 1 ? GPTQ_DQ_RW1 : (nb == 2 ? 4 : 2); }
+__host__ __device__ constexpr int rows_per_warp(int nb) { return nb == 1 ? 8 : (nb == 2 ? 4 : 2); }
 constexpr int kUnitsPerTile = 128;  // 32-column units per column tile of the register form
 
 template <typename T>
