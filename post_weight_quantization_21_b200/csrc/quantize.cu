@@ -206,14 +206,23 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 // rows twice the warps (the step latency needs several warps per scheduler to hide).  The raw U
 // block (B x B) sits in shared memory with each row's C-column chunks padded apart so the group's
 // float4 reads of a row fall in distinct bank groups; err * U[i, j] with err = delta / U_ii is the
-// page's update.
+// page's update.  The block's errors leave as fp32 (err_out), or, for the updates on CTA pairs,
+// already split into tf32 hi = tf32(err) rounded to nearest and lo = tf32(err - hi) (e_hi / e_lo
+// non-null; the same layout, row stride err_ld), which saves a split launch per block.
+__device__ __forceinline__ float tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 template <int C, int LPR>
 __global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, int64_t m, int d, int i1,
                                                       const float* __restrict__ U, int bits,
                                                       int group_size, uint8_t* __restrict__ codes,
                                                       float* __restrict__ scales,
                                                       int32_t* __restrict__ zeros,
-                                                      float* __restrict__ err_out, int err_ld) {
+                                                      float* __restrict__ err_out, int err_ld,
+                                                      float* __restrict__ e_hi, float* __restrict__ e_lo) {
   constexpr int B = LPR * C;
   constexpr int CS = ((C + 4) / 4) % 2 == 1 ? C + 4 : C + 8;  // chunk stride: an odd number of 16-byte granules
   constexpr int RS = LPR * CS;                                  // row stride
@@ -329,10 +338,21 @@ __global__ void __launch_bounds__(128, 3) colloop_kernel(float* __restrict__ w, 
   uint8_t* crow = codes + row * d + i1 + sub * C;
 #pragma unroll
   for (int q = 0; q < C / 4; ++q) reinterpret_cast<uint32_t*>(crow)[q] = cw[q];
-  float* erow = err_out + row * err_ld + sub * C;
+  const int64_t eo = row * err_ld + sub * C;
+  if (e_hi != nullptr) {
 #pragma unroll
-  for (int q = 0; q < C / 4; ++q)
-    *reinterpret_cast<float4*>(erow + 4 * q) = make_float4(er[4 * q], er[4 * q + 1], er[4 * q + 2], er[4 * q + 3]);
+    for (int q = 0; q < C / 4; ++q) {
+      float h[4], l[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) h[t] = tf32_rna(er[4 * q + t]), l[t] = tf32_rna(er[4 * q + t] - h[t]);
+      *reinterpret_cast<float4*>(e_hi + eo + 4 * q) = make_float4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<float4*>(e_lo + eo + 4 * q) = make_float4(l[0], l[1], l[2], l[3]);
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < C / 4; ++q)
+      *reinterpret_cast<float4*>(err_out + eo + 4 * q) = make_float4(er[4 * q], er[4 * q + 1], er[4 * q + 2], er[4 * q + 3]);
+  }
 }
 
 // Whole quantization of 8 rows per CTA in one launch (layers whose U stays in L2): for every block,
@@ -670,19 +690,21 @@ gptq_status run_blocks(float* ww, int64_t m, int d, const float* U, int bits, in
     const int o0 = pair ? i1 / outer * outer : i1;           // start of this block's outer block
     const int slot = i1 - o0;                                 // its column offset in the outer block
     float* err_b = err + slot;                                // this block's errors (row stride err_ld)
+    // on the pair path the column loop writes the errors split into tf32 hi / lo (slot of the outer block)
+    float* eh = pair ? pb->e_hi + slot : nullptr;
+    float* el = pair ? pb->e_lo + slot : nullptr;
     if (lpr8)
       colloop_kernel<C8, 8><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err_b,
-                                                        err_ld);
+                                                        err_ld, eh, el);
     else
       colloop_kernel<C4, 4><<<grid_rows, 128, smem, s>>>(ww, m, d, i1, U, bits, gs, codes, scales, zeros, err_b,
-                                                        err_ld);
+                                                        err_ld, eh, el);
     GPTQ_LAUNCH_CHECK();
     const int rest = d - (i1 + B);
     if (rest > 0) {
       if (pair) {
         const int oend = std::min(o0 + outer, d);
-        gptq_status st = split_rows_launch(err_b, err_ld, m, pb->e_hi + slot, pb->e_lo + slot, kOuter, s);
-        if (st != GPTQ_OK) return st;
+        gptq_status st = GPTQ_OK;
         if (i1 + B < oend) {  // the rest of this outer block, K = 128 (this block's errors)
           CUtensorMap mEbh, mEbl;
           if (!split_map(&mEbh, pb->e_hi + slot, m, B, kOuter) || !split_map(&mEbl, pb->e_lo + slot, m, B, kOuter))
